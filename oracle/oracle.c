@@ -1,0 +1,306 @@
+/*
+ * ORACLE — test infrastructure only.  A plain, slow, obviously correct CPU
+ * implementation of the ExpertsInt8 mixture-of-experts layer, in IEEE fp64
+ * (fp32 where the method fixes fp32).  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library; the CUDA path shares no
+ * code, header, table or helper with it.
+ *
+ * What it computes, and where that is defined:
+ *   - oracle_quantize_rows: ExpertsInt8 weight quantization (Jamba-1.5 paper,
+ *     §3.1 "ExpertsInt8": MoE/MLP weights are quantized to INT8 and stored in
+ *     INT8, without calibration).  Readings of what the page leaves open:
+ *     one fp32 scale per output channel (row of the [out][in] matrix),
+ *     symmetric range [-127, 127], scale = amax / 127 in fp32 round-to-nearest,
+ *     q = round-half-to-even of the exact quotient w / scale (taken in fp64,
+ *     which decides every tie exactly for a bf16 w and an fp32 scale), and an
+ *     all-zero row gets scale 1 and q = 0.
+ *   - oracle_route: the MoE router (Jamba-1.5 paper, "Model Architecture":
+ *     n = 16 experts, the top K = 2 selected at each token).  Readings: logits
+ *     z_e = sum_i x_i * Wr[e][i] (+ bias_e), softmax over all E experts,
+ *     the K largest logits in descending order (equal logits: lower expert
+ *     index first), weights = the softmax probabilities of the chosen experts,
+ *     not renormalised.
+ *   - oracle_moe_forward: y_t = sum_k w_tk * E_{e_tk}(x_t) with SwiGLU experts
+ *     E_e(x) = W2_e (SiLU(W1_e x) * (W3_e x)) (GLU variants, Shazeer 2020,
+ *     cited by the Jamba paper), where each weight is the dequantized value
+ *     q * scale formed exactly in fp64 (Jamba-1.5 paper, §3.1: weights are
+ *     dequantized back before the computation).  No intermediate rounding:
+ *     the result is fp64.
+ *
+ * Parity pins: every function here is checked by the `-m "not gpu"` tests
+ * against exact rational arithmetic, closed forms, invariants and brute-force
+ * special cases that do not reuse this code.
+ *
+ * Build: gcc -O2 -shared -fPIC -pthread oracle.c -lm   (no -ffast-math: the
+ * rounding of every operation must be IEEE round-to-nearest-even).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+/* ---------------------------------------------------------------- helpers */
+
+/* bf16 bit pattern -> the fp32 (hence fp64) value it denotes; exact. */
+static float bf16_value(uint16_t bits) {
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static int pick_threads(int threads, int64_t work_items) {
+    if (threads <= 0) {
+        long n = sysconf(_SC_NPROCESSORS_ONLN);
+        threads = n > 0 ? (int)n : 1;
+    }
+    if (threads > 256) threads = 256;
+    if (work_items < threads) threads = work_items > 0 ? (int)work_items : 1;
+    return threads;
+}
+
+typedef void (*range_fn)(void* ctx, int64_t begin, int64_t end);
+
+typedef struct {
+    range_fn fn;
+    void* ctx;
+    int64_t begin, end;
+} range_job;
+
+static void* range_entry(void* p) {
+    range_job* j = (range_job*)p;
+    j->fn(j->ctx, j->begin, j->end);
+    return NULL;
+}
+
+/* Run fn over [0, n) split into contiguous pieces on `threads` threads. */
+static void parallel_for(int64_t n, int threads, range_fn fn, void* ctx) {
+    threads = pick_threads(threads, n);
+    range_job jobs[256];
+    pthread_t tids[256];
+    int64_t per = (n + threads - 1) / threads;
+    for (int t = 0; t < threads; ++t) {
+        int64_t b = per * t, e = b + per;
+        if (b > n) b = n;
+        if (e > n) e = n;
+        jobs[t] = (range_job){fn, ctx, b, e};
+    }
+    for (int t = 1; t < threads; ++t) pthread_create(&tids[t], NULL, range_entry, &jobs[t]);
+    range_entry(&jobs[0]);
+    for (int t = 1; t < threads; ++t) pthread_join(tids[t], NULL);
+}
+
+/* ------------------------------------------------------------ quantization */
+
+typedef struct {
+    const uint16_t* w;
+    int64_t cols;
+    int8_t* q;
+    float* s;
+} quant_ctx;
+
+/* One output channel: amax, scale = amax/127 (fp32), q = rne(w/scale) in fp64. */
+static void quantize_row(const uint16_t* w, int64_t cols, int8_t* q, float* s) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < cols; ++i) {
+        float a = fabsf(bf16_value(w[i]));
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *s = 1.0f;
+        memset(q, 0, (size_t)cols);
+        return;
+    }
+    const float scale = amax / 127.0f; /* IEEE fp32 division, round to nearest even */
+    *s = scale;
+    for (int64_t i = 0; i < cols; ++i) {
+        double r = nearbyint((double)bf16_value(w[i]) / (double)scale); /* default mode: ties to even */
+        if (r > 127.0) r = 127.0;
+        if (r < -127.0) r = -127.0;
+        q[i] = (int8_t)r;
+    }
+}
+
+static void quantize_range(void* p, int64_t b, int64_t e) {
+    quant_ctx* c = (quant_ctx*)p;
+    for (int64_t r = b; r < e; ++r) quantize_row(c->w + r * c->cols, c->cols, c->q + r * c->cols, c->s + r);
+}
+
+/* w: bf16 bits [rows][cols]; q: int8 [rows][cols]; s: fp32 [rows]. Returns 0, or -1 on bad args. */
+int oracle_quantize_rows(const uint16_t* w, int64_t rows, int64_t cols, int8_t* q, float* s, int threads) {
+    if (!w || !q || !s || rows < 0 || cols <= 0) return -1;
+    quant_ctx c = {w, cols, q, s};
+    parallel_for(rows, threads, quantize_range, &c);
+    return 0;
+}
+
+/* ----------------------------------------------------------------- routing */
+
+/* Logits in fp64, softmax over all E, top-K by logit (ties: lower index first),
+ * weights = chosen probabilities (not renormalised). */
+static void route_token(const uint16_t* x, int64_t d, const float* wr, const float* bias, int E, int K,
+                        int32_t* ids, double* wts, double* logits) {
+    double z[64];
+    for (int e = 0; e < E; ++e) {
+        double acc = 0.0;
+        const float* row = wr + (int64_t)e * d;
+        for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i]) * (double)row[i];
+        if (bias) acc += (double)bias[e];
+        z[e] = acc;
+        if (logits) logits[e] = acc;
+    }
+    double zmax = z[0];
+    for (int e = 1; e < E; ++e)
+        if (z[e] > zmax) zmax = z[e];
+    double p[64], denom = 0.0;
+    for (int e = 0; e < E; ++e) {
+        p[e] = exp(z[e] - zmax);
+        denom += p[e];
+    }
+    for (int e = 0; e < E; ++e) p[e] /= denom;
+    int taken[64] = {0};
+    for (int k = 0; k < K; ++k) {
+        int best = -1;
+        for (int e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || z[e] > z[best]) best = e; /* strict: equal logits keep the lower index */
+        }
+        taken[best] = 1;
+        ids[k] = best;
+        wts[k] = p[best];
+    }
+}
+
+typedef struct {
+    const uint16_t* x;
+    int64_t d;
+    const float* wr;
+    const float* bias;
+    int E, K;
+    int32_t* ids;
+    double* wts;
+    double* logits;
+} route_ctx;
+
+static void route_range(void* p, int64_t b, int64_t e) {
+    route_ctx* c = (route_ctx*)p;
+    for (int64_t t = b; t < e; ++t)
+        route_token(c->x + t * c->d, c->d, c->wr, c->bias, c->E, c->K, c->ids + t * c->K, c->wts + t * c->K,
+                    c->logits ? c->logits + t * c->E : NULL);
+}
+
+/* x: bf16 bits [T][d]; wr: fp32 [E][d]; bias: fp32 [E] or NULL.
+ * ids: int32 [T][K]; wts: fp64 [T][K]; logits: fp64 [T][E] or NULL.  Returns 0, or -1 on bad args. */
+int oracle_route(const uint16_t* x, int64_t T, int64_t d, const float* wr, const float* bias, int E, int K,
+                 int32_t* ids, double* wts, double* logits, int threads) {
+    if (!x || !wr || !ids || !wts || T < 0 || d <= 0 || E < 1 || E > 64 || K < 1 || K > E) return -1;
+    route_ctx c = {x, d, wr, bias, E, K, ids, wts, logits};
+    parallel_for(T, threads, route_range, &c);
+    return 0;
+}
+
+/* ----------------------------------------------------------------- experts */
+
+typedef struct {
+    const uint16_t* x;
+    int64_t d, F;
+    int E, K;
+    const float* wr;
+    const float* bias;
+    const int8_t *q1, *q3, *q2;
+    const float *s1, *s3, *s2;
+    const int64_t* tokens;
+    double* y;
+    int32_t* ids;
+    double* wts;
+    double* h_out;
+} fwd_ctx;
+
+/* One SwiGLU expert on one token with dequantized weights w = q * s (exact in fp64):
+ *   a1_j = sum_i w1[j][i] x_i,  a3_j = sum_i w3[j][i] x_i,
+ *   h_j = SiLU(a1_j) * a3_j = a1_j / (1 + exp(-a1_j)) * a3_j,
+ *   o_i = sum_j w2[i][j] h_j. */
+static void expert_ffn(const fwd_ctx* c, int e, const double* xd, double* h, double* o) {
+    const int64_t d = c->d, F = c->F;
+    const int8_t* q1 = c->q1 + (int64_t)e * F * d;
+    const int8_t* q3 = c->q3 + (int64_t)e * F * d;
+    const int8_t* q2 = c->q2 + (int64_t)e * d * F;
+    const float* s1 = c->s1 + (int64_t)e * F;
+    const float* s3 = c->s3 + (int64_t)e * F;
+    const float* s2 = c->s2 + (int64_t)e * d;
+    for (int64_t j = 0; j < F; ++j) {
+        double a1 = 0.0, a3 = 0.0;
+        const double sc1 = (double)s1[j], sc3 = (double)s3[j];
+        const int8_t* r1 = q1 + j * d;
+        const int8_t* r3 = q3 + j * d;
+        for (int64_t i = 0; i < d; ++i) {
+            a1 += ((double)r1[i] * sc1) * xd[i];
+            a3 += ((double)r3[i] * sc3) * xd[i];
+        }
+        h[j] = a1 / (1.0 + exp(-a1)) * a3;
+    }
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        const double sc2 = (double)s2[i];
+        const int8_t* r2 = q2 + i * F;
+        for (int64_t j = 0; j < F; ++j) acc += ((double)r2[j] * sc2) * h[j];
+        o[i] = acc;
+    }
+}
+
+static void forward_range(void* p, int64_t b, int64_t e) {
+    fwd_ctx* c = (fwd_ctx*)p;
+    const int64_t d = c->d, F = c->F;
+    double* xd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    int32_t ids[64];
+    double wts[64];
+    for (int64_t n = b; n < e; ++n) {
+        const int64_t t = c->tokens ? c->tokens[n] : n;
+        const uint16_t* xt = c->x + t * d;
+        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);
+        route_token(xt, d, c->wr, c->bias, c->E, c->K, ids, wts, NULL);
+        double* yt = c->y + n * d;
+        for (int64_t i = 0; i < d; ++i) yt[i] = 0.0;
+        for (int k = 0; k < c->K; ++k) {
+            expert_ffn(c, ids[k], xd, h, o);
+            for (int64_t i = 0; i < d; ++i) yt[i] += wts[k] * o[i];
+            if (c->h_out) memcpy(c->h_out + (n * c->K + k) * F, h, sizeof(double) * (size_t)F);
+            if (c->ids) c->ids[n * c->K + k] = ids[k];
+            if (c->wts) c->wts[n * c->K + k] = wts[k];
+        }
+    }
+    free(xd);
+    free(h);
+    free(o);
+}
+
+/* The layer on a subset of tokens.
+ *   x: bf16 bits [T][d]; wr fp32 [E][d]; bias fp32 [E] or NULL;
+ *   q1, q3: int8 [E][F][d] with s1, s3 fp32 [E][F]; q2: int8 [E][d][F] with s2 fp32 [E][d];
+ *   tokens: int64 [n_tokens] indices into x, or NULL for tokens 0..n_tokens-1;
+ *   y: fp64 [n_tokens][d] (output);
+ *   ids int32 [n_tokens][K], wts fp64 [n_tokens][K], h_out fp64 [n_tokens][K][F]: optional outputs.
+ * Returns 0, or -1 on bad arguments. */
+int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t d, int64_t F, int E, int K, const float* wr,
+                       const float* bias, const int8_t* q1, const float* s1, const int8_t* q3, const float* s3,
+                       const int8_t* q2, const float* s2, const int64_t* tokens, int64_t n_tokens, double* y,
+                       int32_t* ids, double* wts, double* h_out, int threads) {
+    if (!x || !wr || !q1 || !s1 || !q3 || !s3 || !q2 || !s2 || !y) return -1;
+    if (T < 0 || d <= 0 || F <= 0 || E < 1 || E > 64 || K < 1 || K > E || n_tokens < 0) return -1;
+    if (tokens) {
+        for (int64_t n = 0; n < n_tokens; ++n)
+            if (tokens[n] < 0 || tokens[n] >= T) return -1;
+    } else if (n_tokens > T) {
+        return -1;
+    }
+    fwd_ctx c = {x, d, F, E, K, wr, bias, q1, q3, q2, s1, s3, s2, tokens, y, ids, wts, h_out};
+    parallel_for(n_tokens, threads, forward_range, &c);
+    return 0;
+}
+
+/* Number of host threads the oracle uses when asked for "all" (threads <= 0). */
+int oracle_default_threads(void) { return pick_threads(0, 1 << 30); }
