@@ -1,0 +1,429 @@
+"""Benchmark of the ExpertsInt8 MoE layer (tokens/s through jamba_moe_forward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one forward pass of the whole layer (router, permutation, expert GEMMs with in-kernel
+int8 -> bf16 dequantization, weighted combine) over one batch of T synthetic tokens.  The int8
+weights are quantized once, before timing (load time), by the library's quantize kernel, which is
+timed on its own and reported under "quantize".  Under torchrun every rank runs its own batch with
+replicated weights (weak scaling, no collective on the data path); the time is the max over ranks.
+
+Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle on bounded samples of the
+same workload on the host cores (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/sec (int8 experts) at 1 B200; % of HBM / BF16 roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "v01_decode"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ------------------------------------------------------------------ algorithmic work per launch
+def algorithmic(kind, wl, T, touched, rows_padded):
+    """Bytes (HBM-bound kernels) or FLOPs (tensor-bound kernels) one launch must move / do.
+    touched = experts with >= 1 token; rows_padded = permuted rows incl. per-expert padding."""
+    d, F, TK = wl.d, wl.F, T * wl.K
+    if kind == "gemv13":
+        return "bytes", touched * (2 * F * d + 2 * F * 4) + TK * d * 2 + TK * F * 2
+    if kind == "gemv2":
+        return "bytes", touched * (d * F + d * 4) + TK * F * 2 + TK * d * 4 + TK * 4 * 2
+    if kind == "gemm13":
+        return "flops", 2.0 * TK * d * (2 * F)
+    if kind == "gemm2":
+        return "flops", 2.0 * TK * F * d
+    if kind == "combine":
+        return "bytes", TK * d * 4 + T * d * 2
+    if kind == "router":
+        return "bytes", T * d * 2 + wl.E * d * 4 + TK * 8
+    if kind == "gather":
+        return "bytes", rows_padded * d * 2 + TK * d * 2
+    if kind == "permute":
+        return "bytes", TK * 4 * 3
+    if kind == "quantize":
+        return "bytes", 3 * (2 * F * d + d * F) * wl.E
+    return "bytes", 0
+
+
+def kernel_source_hash(kind):
+    files = {"gemv13": ["gemv.cu"], "gemv2": ["gemv.cu"], "gemm13": ["gemm_tc.cu"], "gemm2": ["gemm_tc.cu"],
+             "quantize": ["quantize.cu"], "router": ["router.cu"], "combine": ["combine.cu"],
+             "permute": ["permute.cu"], "gather": ["permute.cu"]}.get(kind, [])
+    h = hashlib.sha256()
+    for f in files + ["common.cuh"]:
+        p = os.path.join(ROOT, "int8_expert_weight_b200", "csrc", f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kind, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    rec = json.load(open(p)).get(f"{kind}@{workload}")
+    if not rec or rec.get("source_sha256") != kernel_source_hash(kind):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ clocks during the timed region
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out" if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ".",
+                                 f".clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[4]), parts[5:]))
+            except ValueError:
+                continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [r for r in rows if r[2] > 0] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(loaded)}
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+def oracle_setup(wl, seed_x):
+    """Host copies for the oracle: bf16 x, router, and the oracle's own quantization of the weights."""
+    import oracle
+    x = synth.gen_x(synth_replace(wl, seed=seed_x))
+    wr = synth.gen_router(wl)
+    bias = synth.gen_bias(wl)
+    qs = {}
+    for which in ("w1", "w3", "w2"):
+        rows, cols = synth.weight_shape(wl, which)
+        q = np.empty((wl.E, rows, cols), np.int8)
+        s = np.empty((wl.E, rows), np.float32)
+        for e in range(wl.E):
+            q[e], s[e] = oracle.quantize(synth.gen_expert(wl, which, e))
+        qs[which] = (q, s)
+    return x, wr, bias, qs
+
+
+def synth_replace(wl, **kw):
+    import dataclasses
+    return dataclasses.replace(wl, **kw)
+
+
+def oracle_rate(wl, setup, budget_s, max_tokens=None):
+    """Tokens/s of the oracle forward on a bounded sample (tokens spread over the batch)."""
+    import oracle
+    x, wr, bias, qs = setup
+    threads = oracle.default_threads()
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=[0], threads=1)
+    per_token_1t = time.perf_counter() - t0
+    n = max(1, min(wl.T, int(budget_s * threads / max(per_token_1t, 1e-9))))
+    if max_tokens:
+        n = min(n, max_tokens)
+    toks = np.linspace(0, wl.T - 1, n).round().astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+    dt = time.perf_counter() - t0
+    used = min(threads, n)
+    return n / dt, used, n, dt
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[args.workload]
+    setup = oracle_setup(wl, wl.seed)
+    import oracle
+    threads = oracle.default_threads()
+    # calibrate one token on one thread, then size every step to fit a few minutes in total
+    x, wr, bias, qs = setup
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=[0], threads=1)
+    per_tok = time.perf_counter() - t0
+    step_budget = min(args.cpu_budget_s, 150.0 / max(1, args.steps + args.warmup))
+    n = int(max(1, min(wl.T, step_budget * threads / per_tok)))
+    toks = np.linspace(0, wl.T - 1, n).round().astype(np.int64)
+    for _ in range(args.warmup):
+        oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    sample = f"{n} of {wl.T} tokens per step (evenly spaced), full fp64 layer per token"
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": workload_config(wl, "oracle"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, n), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    return 0
+
+
+def workload_config(wl, path):
+    return {"workload": wl.name, "T": wl.T, "d": wl.d, "ffn": wl.F, "experts": wl.E, "top_k": wl.K,
+            "weights": "int8 codes + fp32 per-output-channel scales", "activations": "bf16",
+            "path": path, "l2": l2_note(wl)}
+
+
+def l2_note(wl):
+    wbytes = 3 * wl.E * wl.d * wl.F
+    if wbytes > 126e6:
+        return "inputs larger than L2: int8 expert weights %.2f GB > 126 MB L2, no flush" % (wbytes / 1e9)
+    return "inputs fit in L2 (%.1f MB): not a roofline workload" % (wbytes / 1e6)
+
+
+# ------------------------------------------------------------------ the CUDA arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import int8_expert_weight_b200 as jm
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    wl = synth.WORKLOADS[args.workload]
+    T, d, F, E = wl.T, wl.d, wl.F, wl.E
+    path = {"auto": jm.PATH_AUTO, "gemv": jm.PATH_GEMV, "gemm": jm.PATH_GEMM}[args.path]
+    peaks = load_peaks()
+
+    # ---- inputs: this rank's batch (own seed), replicated weights quantized by the library (load time)
+    seed_x = wl.seed + rank
+    x_bits = synth.gen_x(synth_replace(wl, seed=seed_x))
+    to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa
+    x = to_dev(x_bits)
+    wr = torch.from_numpy(synth.gen_router(wl)).to(dev)
+    bias_np = synth.gen_bias(wl)
+    bias = None if bias_np is None else torch.from_numpy(bias_np).to(dev)
+    Q, S = {}, {}
+    q_ms = 0.0
+    qe0, qe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for which in ("w1", "w3", "w2"):
+        rows, cols = synth.weight_shape(wl, which)
+        Q[which] = torch.empty((E, rows, cols), dtype=torch.int8, device=dev)
+        S[which] = torch.empty((E, rows), dtype=torch.float32, device=dev)
+        for e in range(E):
+            w = to_dev(synth.gen_expert(wl, which, e))
+            qe0.record()
+            jm.jamba_moe_quantize(w, out=(Q[which][e], S[which][e]))
+            qe1.record()
+            torch.cuda.synchronize()
+            q_ms += qe0.elapsed_time(qe1)
+            del w
+    q_bytes = algorithmic("quantize", wl, T, 0, 0)[1]
+    ws = torch.empty(jm.jamba_moe_workspace_size(T, d, F), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    ids = torch.empty((T, 2), dtype=torch.int32, device=dev)
+    tw = torch.empty((T, 2), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        jm.jamba_moe_forward(x, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y, topk_ids=ids,
+                             topk_w=tw, workspace=ws, path=path)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = jm.jamba_moe_read_device_status(ws)
+    ids_np = ids.cpu().numpy()
+    touched = int(np.unique(ids_np).size)
+    counts = np.bincount(ids_np.reshape(-1), minlength=E)
+    rows_padded = int(sum((c + 127) // 128 * 128 for c in counts))
+
+    # ---- timed region: K forward steps on resident inputs, per-kernel events recorded live
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local_rank) as clk:
+        jm.jamba_moe_timing_start(args.steps * 16)
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        kernels = jm.jamba_moe_timing_collect()
+        jm.jamba_moe_timing_start(0)
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    value = world * T * args.steps / (ms / 1e3)
+
+    # ---- end to end through the public call with host buffers: pinned x in, pinned y out
+    x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    x_host.copy_(x.cpu())
+    y_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
+    x_dev = torch.empty_like(x)
+
+    def step_e2e():
+        x_dev.copy_(x_host, non_blocking=True)
+        jm.jamba_moe_forward(x_dev, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
+                             topk_ids=ids, topk_w=tw, workspace=ws, path=path)
+        y_host.copy_(y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step_e2e()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step_e2e()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+
+    # ---- roofline of the dominant kernel
+    dom = max(kernels, key=lambda k: kernels[k][0])
+    dom_ms, dom_n = kernels[dom]
+    unit_kind, work = algorithmic(dom, wl, T, touched, rows_padded)
+    avg_s = dom_ms / dom_n / 1e3
+    if unit_kind == "bytes":
+        achieved, peak, unit, bound = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+    else:
+        achieved, peak, unit, bound = work / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s", "tensor"
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                "traffic": ncu_traffic(dom, wl.name), "kernel": dom, "algorithmic_per_launch": work,
+                "peak_source": peaks["source"]}
+    per_kernel = {}
+    for k, (kms, n) in sorted(kernels.items(), key=lambda kv: -kv[1][0]):
+        uk, wk = algorithmic(k, wl, T, touched, rows_padded)
+        a = wk / (kms / n / 1e3)
+        per_kernel[k] = {"launches": n, "avg_us": kms / n * 1e3,
+                         ("GB/s" if uk == "bytes" else "TFLOP/s"): a / (1e9 if uk == "bytes" else 1e12)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        setup = oracle_setup(wl, seed_x)
+        rate, cores, n, dt = oracle_rate(wl, setup, args.cpu_budget_s)
+        cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{n} of {wl.T} tokens (evenly spaced) of the same batch, fp64, {dt:.1f} s"}
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu"),
+            "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
+                    "d2h_bytes_per_step": T * d * 2},
+            "gpu_launches": int(sum(n for _, n in kernels.values())),
+            "clocks": clk.summary(), "kernels": per_kernel, "device_status": status,
+            "routing": {"touched_experts": touched, "max_tokens_per_expert": int(counts.max())},
+            "quantize": {"ms": q_ms, "GB/s": q_bytes / (q_ms / 1e3) / 1e9,
+                         "frac_of_hbm": q_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+        }
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,164 @@
+/*
+ * jmoe.h — C ABI of the ExpertsInt8 mixture-of-experts layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (Jamba-1.5: Hybrid Transformer-Mamba Models at Scale, "Model Architecture":
+ * n = 16 experts, the top K = 2 chosen at each token; §3.1 "ExpertsInt8": expert weights are
+ * quantized to INT8, stored in INT8 and turned back into BF16 inside the fused MoE kernel,
+ * right before the matrix math) computes, for every token x_t (a row of d bf16 values):
+ *
+ *     z_e   = sum_i x_ti * Wr[e][i] (+ b_e)                  router logits, fp32
+ *     p     = softmax(z)                                      over all 16 experts
+ *     e_t1, e_t2 = the two largest logits, in descending order
+ *     y_t   = p_{e_t1} * E_{e_t1}(x_t) + p_{e_t2} * E_{e_t2}(x_t)   (weights not renormalised)
+ *     E_e(x) = W2_e ( SiLU(W1_e x) * (W3_e x) )               SwiGLU expert
+ *
+ * with W1_e, W3_e: [ffn][d] and W2_e: [d][ffn] held as int8 codes Q plus one fp32 scale S per
+ * output row (W[r][c] ~= Q[r][c] * S[r]).
+ *
+ * Conventions for every call below
+ *   - "bf16" buffers are arrays of uint16_t holding bfloat16 bit patterns.
+ *   - Every pointer is a DEVICE pointer owned by the caller, unless a comment says otherwise.
+ *     The library allocates no device memory, never synchronises the stream (except where
+ *     stated) and launches its kernels only on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).
+ *   - Tensors are dense, row-major, with the last dimension contiguous.  Device pointers must
+ *     be 16-byte aligned.
+ *   - Calls return a jmoe_status.  Argument errors are detected on the host before anything is
+ *     launched and leave all buffers untouched.  Launch failures return JMOE_ERR_CUDA.  No call
+ *     aborts, throws or prints.
+ *   - Calls are asynchronous: results are ready when `stream` reaches the point of the call.
+ *   - Supported shapes: n_experts == 16, top_k == 2, d and ffn multiples of 128 with
+ *     128 <= d, ffn <= 32768, 1 <= T <= 1048576.  Anything else returns JMOE_ERR_SHAPE.
+ */
+#ifndef JMOE_H
+#define JMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    JMOE_OK = 0,
+    JMOE_ERR_NULL = 1,       /* a required pointer is NULL */
+    JMOE_ERR_SHAPE = 2,      /* unsupported or inconsistent sizes */
+    JMOE_ERR_WORKSPACE = 3,  /* workspace too small or misaligned */
+    JMOE_ERR_CUDA = 4,       /* a CUDA runtime call or kernel launch failed */
+    JMOE_DEV_TIMEOUT = 5,    /* a kernel gave up waiting on a pipeline barrier (device status) */
+    JMOE_DEV_BAD_INDEX = 6,  /* a kernel saw an out-of-range routing index (device status) */
+    JMOE_ERR_ALIGN = 7       /* a pointer is not 16-byte aligned */
+} jmoe_status;
+
+/* Forward-path selection for jamba_moe_forward_path. */
+enum {
+    JMOE_PATH_AUTO = 0,  /* decode GEMV path when T <= 128, grouped tensor-core GEMM otherwise */
+    JMOE_PATH_GEMV = 1,  /* weight-streaming path for few tokens per expert */
+    JMOE_PATH_GEMM = 2   /* tcgen05 grouped GEMM path (prefill) */
+};
+
+/*
+ * jamba_moe_quantize — ExpertsInt8 weight quantization (Jamba-1.5 paper, §3.1: weights are
+ * quantized to INT8 at model loading, without calibration).
+ *
+ *   W: bf16 [n_mats][rows][cols]   input weights, out x in (one row per output channel)
+ *   Q: int8 [n_mats][rows][cols]   output codes
+ *   S: fp32 [n_mats][rows]         output scales, one per row
+ *
+ * For each row r: amax = max_c |W[r][c]|; S[r] = amax / 127 (fp32, round to nearest even);
+ * Q[r][c] = the integer nearest to W[r][c] / S[r] (exact quotient; halfway cases to even),
+ * within [-127, 127].  A row of zeros gets S = 1 and Q = 0.  The scale granularity (per output
+ * channel), the symmetric range and the rounding rule are this library's reading of what the
+ * page leaves open.  Results are bit-exact and deterministic.
+ * Sizes: n_mats >= 1, 1 <= rows, 16 <= cols <= 1<<20 with cols % 16 == 0; W, Q 16-byte aligned.
+ */
+int jamba_moe_quantize(const uint16_t* W, int64_t n_mats, int64_t rows, int64_t cols, int8_t* Q, float* S,
+                       void* stream);
+
+/*
+ * jamba_moe_workspace_size — bytes of device scratch jamba_moe_forward needs for these sizes
+ * (routing tables, the permuted activations, the SwiGLU intermediate and the per-slot
+ * outputs).  Returns 0 for unsupported sizes.  Host only; touches no device.
+ */
+size_t jamba_moe_workspace_size(int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k);
+
+/*
+ * jamba_moe_forward — the MoE layer on T tokens (formula at the top of this file).
+ *
+ *   x:           bf16 [T][d]                 activations
+ *   router_W:    fp32 [n_experts][d]         router weight
+ *   router_bias: fp32 [n_experts] or NULL    added to the logits (NULL = no bias)
+ *   Q1, Q3:      int8 [n_experts][ffn][d]    with S1, S3 fp32 [n_experts][ffn]  (gate, up)
+ *   Q2:          int8 [n_experts][d][ffn]    with S2 fp32 [n_experts][d]        (down)
+ *   y:           bf16 [T][d]                 output (written)
+ *   topk_ids:    int32 [T][top_k] or NULL    chosen experts, descending logit (written if given)
+ *   topk_w:      fp32 [T][top_k] or NULL     their softmax probabilities (written if given)
+ *   workspace:   device scratch of at least jamba_moe_workspace_size(...) bytes, 256-byte
+ *                aligned, owned by the caller; its contents on entry do not matter.  One
+ *                workspace must not be used by two calls that may overlap on the GPU.
+ *
+ * Numerics: router in fp32; int8 codes converted exactly to bf16 inside the GEMM kernels,
+ * bf16 x bf16 products accumulated in fp32, per-row scales applied to the fp32 accumulators;
+ * the SwiGLU intermediate is rounded to bf16; the two weighted expert outputs of a token are
+ * added in fp32 in a fixed order (slot 0 then slot 1) and rounded once to bf16.  The result
+ * is deterministic (no floating-point atomics).  Experts that receive no token are skipped and
+ * their weights are not read.
+ */
+int jamba_moe_forward(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
+                      const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,
+                      int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y,
+                      int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * jamba_moe_forward_path — jamba_moe_forward with the expert-GEMM path chosen explicitly
+ * (JMOE_PATH_*).  Both paths compute the same function; tests use this to run each path on
+ * every shape.  An unknown path value returns JMOE_ERR_SHAPE.
+ */
+int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float* router_bias,
+                           const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                           const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, int n_experts,
+                           int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w, void* workspace,
+                           size_t workspace_bytes, void* stream, int path);
+
+/*
+ * jamba_moe_read_device_status — synchronises `stream`, then returns the status word the
+ * kernels of the last forward call on `workspace` left there: JMOE_OK, JMOE_DEV_TIMEOUT (a
+ * pipeline wait ran out of its bounded number of polls; the kernel released its resources and
+ * returned early, so y is not valid) or JMOE_DEV_BAD_INDEX.  JMOE_ERR_CUDA if the copy fails.
+ */
+int jamba_moe_read_device_status(const void* workspace, void* stream);
+
+/* jamba_moe_status_string — static, human-readable text for a jmoe_status value (host only). */
+const char* jamba_moe_status_string(int status);
+
+/*
+ * Kernel timing (for the benchmark's roofline figures).
+ * jamba_moe_timing_start(max_launches) makes every following launch of this library record a
+ * pair of CUDA events on its stream, until max_launches pairs are recorded, and forgets any
+ * earlier records; max_launches <= 0 switches recording off.  jamba_moe_timing_collect
+ * synchronises those events and writes, for each kernel kind k < n_kinds (JMOE_KERNEL_*),
+ * total_ms[k] (sum of event-measured durations) and launches[k]; it returns the number of
+ * kinds written.  Host pointers.  Not thread-safe: one timing session per process.
+ */
+enum {
+    JMOE_KERNEL_QUANTIZE = 0,
+    JMOE_KERNEL_ROUTER = 1,
+    JMOE_KERNEL_PERMUTE = 2,
+    JMOE_KERNEL_GATHER = 3,
+    JMOE_KERNEL_GEMV13 = 4,
+    JMOE_KERNEL_GEMV2 = 5,
+    JMOE_KERNEL_GEMM13 = 6,
+    JMOE_KERNEL_GEMM2 = 7,
+    JMOE_KERNEL_COMBINE = 8,
+    JMOE_KERNEL_KINDS = 9
+};
+int jamba_moe_timing_start(int max_launches);
+int jamba_moe_timing_collect(double* total_ms, int64_t* launches, int n_kinds);
+const char* jamba_moe_kernel_name(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JMOE_H */

@@ -1,0 +1,194 @@
+"""ExpertsInt8 mixture-of-experts layer for NVIDIA B200 — thin Python binding of libjmoe.so.
+
+Every step of the layer runs in the CUDA kernels of ``libjmoe.so`` (see ``include/jmoe.h`` for
+the C ABI).  This module only marshals arguments: it checks dtypes, devices and shapes of torch
+tensors, passes their device pointers and the current CUDA stream, and turns a non-zero status
+into a ``JmoeError``.  PyTorch provides device memory and streams; there is no CPU path.
+
+Functions keep the C names: ``jamba_moe_quantize``, ``jamba_moe_workspace_size``,
+``jamba_moe_forward``, ``jamba_moe_read_device_status``, ``jamba_moe_status_string``,
+``jamba_moe_timing_start``, ``jamba_moe_timing_collect``.
+"""
+import ctypes
+import os
+from typing import Dict, Optional, Tuple
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libjmoe.so")
+
+N_EXPERTS = 16
+TOP_K = 2
+PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
+KERNEL_NAMES = ["quantize", "router", "permute", "gather", "gemv13", "gemv2", "gemm13", "gemm2", "combine"]
+
+
+class JmoeError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {jamba_moe_status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libjmoe.so; raises if it has not been built (run int8_expert_weight_b200/build.py)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libjmoe.so not found at {path}: build it with `python int8_expert_weight_b200/build.py`")
+    lib = ctypes.CDLL(path)
+    vp, i64, c_int, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.jamba_moe_quantize.restype = c_int
+    lib.jamba_moe_quantize.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+    lib.jamba_moe_workspace_size.restype = sz
+    lib.jamba_moe_workspace_size.argtypes = [i64, i64, i64, c_int, c_int]
+    fwd_args = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, sz, vp]
+    lib.jamba_moe_forward.restype = c_int
+    lib.jamba_moe_forward.argtypes = fwd_args
+    lib.jamba_moe_forward_path.restype = c_int
+    lib.jamba_moe_forward_path.argtypes = fwd_args + [c_int]
+    lib.jamba_moe_read_device_status.restype = c_int
+    lib.jamba_moe_read_device_status.argtypes = [vp, vp]
+    lib.jamba_moe_status_string.restype = ctypes.c_char_p
+    lib.jamba_moe_status_string.argtypes = [c_int]
+    lib.jamba_moe_timing_start.restype = c_int
+    lib.jamba_moe_timing_start.argtypes = [c_int]
+    lib.jamba_moe_timing_collect.restype = c_int
+    lib.jamba_moe_timing_collect.argtypes = [vp, vp, c_int]
+    lib.jamba_moe_kernel_name.restype = ctypes.c_char_p
+    lib.jamba_moe_kernel_name.argtypes = [c_int]
+    _lib = lib
+    return lib
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def jamba_moe_status_string(status: int) -> str:
+    return load_library().jamba_moe_status_string(int(status)).decode()
+
+
+def jamba_moe_workspace_size(T: int, d: int, ffn: int, n_experts: int = N_EXPERTS, top_k: int = TOP_K) -> int:
+    return int(load_library().jamba_moe_workspace_size(T, d, ffn, n_experts, top_k))
+
+
+def jamba_moe_quantize(W: torch.Tensor, stream: Optional[torch.cuda.Stream] = None,
+                       out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """ExpertsInt8 quantization of bf16 weights [..., rows, cols] (one scale per row).
+    Returns (Q int8 same shape, S fp32 shape[:-1])."""
+    lib = load_library()
+    _check(W, "W", torch.bfloat16)
+    if W.dim() < 2:
+        raise ValueError("W must have at least 2 dims (rows, cols)")
+    rows, cols = W.shape[-2], W.shape[-1]
+    n_mats = W.numel() // (rows * cols) if W.numel() else 0
+    if out is None:
+        Q = torch.empty(W.shape, dtype=torch.int8, device=W.device)
+        S = torch.empty(W.shape[:-1], dtype=torch.float32, device=W.device)
+    else:
+        Q, S = out
+        _check(Q, "Q", torch.int8, W.shape)
+        _check(S, "S", torch.float32, W.shape[:-1])
+    st = lib.jamba_moe_quantize(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(), _stream_ptr(stream))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_quantize")
+    return Q, S
+
+
+def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor],
+                      Q1: torch.Tensor, S1: torch.Tensor, Q3: torch.Tensor, S3: torch.Tensor,
+                      Q2: torch.Tensor, S2: torch.Tensor, y: Optional[torch.Tensor] = None,
+                      topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                      path: int = PATH_AUTO, want_routing: bool = True):
+    """The MoE layer on x [T][d] (bf16).  Weights as produced by jamba_moe_quantize:
+    Q1, Q3 int8 [16][ffn][d] with S1, S3 fp32 [16][ffn]; Q2 int8 [16][d][ffn] with S2 fp32 [16][d];
+    router_W fp32 [16][d]; router_bias fp32 [16] or None.
+
+    Returns (y bf16 [T][d], topk_ids int32 [T][2] or None, topk_w fp32 [T][2] or None).
+    ``workspace`` (uint8, >= jamba_moe_workspace_size bytes) is allocated when not given.
+    """
+    lib = load_library()
+    _check(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be [T][d]")
+    T, d = x.shape
+    E = router_W.shape[0]
+    ffn = Q1.shape[1]
+    _check(router_W, "router_W", torch.float32, (E, d))
+    if router_bias is not None:
+        _check(router_bias, "router_bias", torch.float32, (E,))
+    _check(Q1, "Q1", torch.int8, (E, ffn, d))
+    _check(Q3, "Q3", torch.int8, (E, ffn, d))
+    _check(Q2, "Q2", torch.int8, (E, d, ffn))
+    _check(S1, "S1", torch.float32, (E, ffn))
+    _check(S3, "S3", torch.float32, (E, ffn))
+    _check(S2, "S2", torch.float32, (E, d))
+    if y is None:
+        y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device)
+    _check(y, "y", torch.bfloat16, (T, d))
+    if want_routing:
+        if topk_ids is None:
+            topk_ids = torch.empty((T, TOP_K), dtype=torch.int32, device=x.device)
+        if topk_w is None:
+            topk_w = torch.empty((T, TOP_K), dtype=torch.float32, device=x.device)
+    if topk_ids is not None:
+        _check(topk_ids, "topk_ids", torch.int32, (T, TOP_K))
+    if topk_w is not None:
+        _check(topk_w, "topk_w", torch.float32, (T, TOP_K))
+    need = jamba_moe_workspace_size(T, d, ffn, E, TOP_K)
+    if need == 0:
+        raise JmoeError(2, "jamba_moe_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    st = lib.jamba_moe_forward_path(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
+                                    S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
+                                    T, d, ffn, E, TOP_K, y.data_ptr(), p(topk_ids), p(topk_w),
+                                    workspace.data_ptr(), workspace.numel(), _stream_ptr(stream), int(path))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_forward")
+    return y, topk_ids, topk_w
+
+
+def jamba_moe_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream and return the device status word of the last forward on workspace."""
+    _check(workspace, "workspace", torch.uint8)
+    return int(load_library().jamba_moe_read_device_status(workspace.data_ptr(), _stream_ptr(stream)))
+
+
+def jamba_moe_timing_start(max_launches: int) -> None:
+    st = load_library().jamba_moe_timing_start(int(max_launches))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_timing_start")
+
+
+def jamba_moe_timing_collect() -> Dict[str, Tuple[float, int]]:
+    """{kernel name: (total event-timed ms, launches)} for the launches recorded since timing_start."""
+    n = len(KERNEL_NAMES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    r = load_library().jamba_moe_timing_collect(ctypes.addressof(ms), ctypes.addressof(cnt), n)
+    if r < 0:
+        raise JmoeError(-r, "jamba_moe_timing_collect")
+    return {KERNEL_NAMES[k]: (ms[k], cnt[k]) for k in range(n) if cnt[k]}

@@ -1,0 +1,274 @@
+// C ABI of the ExpertsInt8 MoE layer: argument checks, workspace layout, kernel sequencing and
+// the optional per-launch event timing.  Declared in include/jmoe.h.
+#include <vector>
+
+#include "common.cuh"
+
+namespace jmoe {
+
+cudaError_t launch_quantize(const uint16_t* W, int64_t rows, int64_t cols, int8_t* Q, float* S, cudaStream_t st,
+                            int num_sms);
+cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int64_t T, int64_t d,
+                          int32_t* ids_ws, float* w_ws, int32_t* ids_user, float* w_user, cudaStream_t st);
+cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
+                           cudaStream_t st);
+cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
+                          uint16_t* x_perm, cudaStream_t st, int num_sms);
+cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
+                          const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
+                          int64_t F, cudaStream_t st);
+cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
+                         const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
+                         cudaStream_t st);
+cudaError_t launch_combine(const float* slots, int64_t T, int64_t d, uint16_t* y, cudaStream_t st, int num_sms);
+
+namespace {
+
+constexpr int64_t kMaxT = int64_t(1) << 20;
+constexpr int64_t kMaxDim = 32768;
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Layout {
+    int64_t rows_cap;  // permuted rows incl. per-expert padding
+    size_t hdr, ids, wts, inv, perm, x_perm, h, slots, total;
+};
+
+bool shape_ok(int64_t T, int64_t d, int64_t F, int E, int K) {
+    if (E != kExperts || K != kTopK) return false;
+    if (T < 1 || T > kMaxT) return false;
+    if (d < 128 || d > kMaxDim || d % 128 != 0) return false;
+    if (F < 128 || F > kMaxDim || F % 128 != 0) return false;
+    return true;
+}
+
+Layout make_layout(int64_t T, int64_t d, int64_t F) {
+    Layout L{};
+    const int64_t TK = T * kTopK;
+    L.rows_cap = (TK + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
+    size_t off = 0;
+    L.hdr = off;
+    off = align256(off + kHeaderBytes);
+    L.ids = off;
+    off = align256(off + sizeof(int32_t) * TK);
+    L.wts = off;
+    off = align256(off + sizeof(float) * TK);
+    L.inv = off;
+    off = align256(off + sizeof(int32_t) * TK);
+    L.perm = off;
+    off = align256(off + sizeof(int32_t) * L.rows_cap);
+    L.x_perm = off;
+    off = align256(off + sizeof(uint16_t) * L.rows_cap * d);
+    L.h = off;
+    off = align256(off + sizeof(uint16_t) * L.rows_cap * F);
+    L.slots = off;
+    off = align256(off + sizeof(float) * TK * d);
+    L.total = off;
+    return L;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int num_sms_current() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// ---------------------------------------------------------------- launch timing
+struct Timing {
+    std::vector<cudaEvent_t> start, stop;
+    std::vector<int> kind;
+    int used = 0;
+    bool on = false;
+} g_timing;
+
+struct TimedLaunch {
+    cudaStream_t st;
+    int slot = -1;
+    TimedLaunch(int kind, cudaStream_t s) : st(s) {
+        if (g_timing.on && g_timing.used < (int)g_timing.start.size()) {
+            slot = g_timing.used++;
+            g_timing.kind[slot] = kind;
+            cudaEventRecord(g_timing.start[slot], st);
+        }
+    }
+    ~TimedLaunch() {
+        if (slot >= 0) cudaEventRecord(g_timing.stop[slot], st);
+    }
+};
+
+int to_status(cudaError_t e) { return e == cudaSuccess ? JMOE_OK : JMOE_ERR_CUDA; }
+
+}  // namespace
+}  // namespace jmoe
+
+using namespace jmoe;
+
+extern "C" {
+
+int jamba_moe_quantize(const uint16_t* W, int64_t n_mats, int64_t rows, int64_t cols, int8_t* Q, float* S,
+                       void* stream) {
+    if (!W || !Q || !S) return JMOE_ERR_NULL;
+    if (n_mats < 1 || rows < 1 || cols < 16 || cols > (int64_t(1) << 20) || cols % 16 != 0) return JMOE_ERR_SHAPE;
+    if (n_mats > (int64_t(1) << 40) / rows) return JMOE_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(Q) || (reinterpret_cast<uintptr_t>(S) & 3)) return JMOE_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TimedLaunch t(JMOE_KERNEL_QUANTIZE, st);
+    return to_status(launch_quantize(W, n_mats * rows, cols, Q, S, st, num_sms_current()));
+}
+
+size_t jamba_moe_workspace_size(int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k) {
+    if (!shape_ok(T, d, ffn, n_experts, top_k)) return 0;
+    return make_layout(T, d, ffn).total;
+}
+
+int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
+                           const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,
+                           int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y,
+                           int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream,
+                           int path) {
+    if (!x || !router_W || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
+    if (!shape_ok(T, d, ffn, n_experts, top_k)) return JMOE_ERR_SHAPE;
+    if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    const void* ptrs16[] = {x, Q1, Q3, Q2, y, router_W};
+    for (const void* p : ptrs16)
+        if (!aligned16(p)) return JMOE_ERR_ALIGN;
+    const void* ptrs4[] = {router_bias, S1, S3, S2, topk_ids, topk_w};
+    for (const void* p : ptrs4)
+        if (reinterpret_cast<uintptr_t>(p) & 3) return JMOE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return JMOE_ERR_WORKSPACE;
+    const Layout L = make_layout(T, d, ffn);
+    if (workspace_bytes < L.total) return JMOE_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+    int32_t* ids = reinterpret_cast<int32_t*>(ws + L.ids);
+    float* wts = reinterpret_cast<float*>(ws + L.wts);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    float* slots = reinterpret_cast<float*>(ws + L.slots);
+    (void)x_perm;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = num_sms_current();
+    if (path == JMOE_PATH_AUTO) path = JMOE_PATH_GEMV;
+    if (path == JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;  // grouped tensor-core path not built yet
+
+    cudaError_t e;
+    {
+        TimedLaunch t(JMOE_KERNEL_ROUTER, st);
+        e = launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
+        e = launch_permute(ids, T, hdr, perm, inv, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_GEMV13, st);
+        e = launch_gemv13(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_GEMV2, st);
+        e = launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_COMBINE, st);
+        e = launch_combine(slots, T, d, y, st, sms);
+    }
+    return to_status(e);
+}
+
+int jamba_moe_forward(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
+                      const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,
+                      int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids,
+                      float* topk_w, void* workspace, size_t workspace_bytes, void* stream) {
+    return jamba_moe_forward_path(x, router_W, router_bias, Q1, S1, Q3, S3, Q2, S2, T, d, ffn, n_experts, top_k, y,
+                                  topk_ids, topk_w, workspace, workspace_bytes, stream, JMOE_PATH_AUTO);
+}
+
+int jamba_moe_read_device_status(const void* workspace, void* stream) {
+    if (!workspace) return JMOE_ERR_NULL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t status = 0;
+    if (cudaMemcpyAsync(&status, workspace, sizeof(status), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return JMOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return JMOE_ERR_CUDA;
+    return (int)status;
+}
+
+const char* jamba_moe_status_string(int status) {
+    switch (status) {
+        case JMOE_OK: return "ok";
+        case JMOE_ERR_NULL: return "a required pointer is NULL";
+        case JMOE_ERR_SHAPE: return "unsupported or inconsistent sizes";
+        case JMOE_ERR_WORKSPACE: return "workspace too small or not 256-byte aligned";
+        case JMOE_ERR_CUDA: return "CUDA runtime call or kernel launch failed";
+        case JMOE_DEV_TIMEOUT: return "a kernel gave up waiting on a pipeline barrier";
+        case JMOE_DEV_BAD_INDEX: return "a kernel saw an out-of-range routing index";
+        case JMOE_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        default: return "unknown status";
+    }
+}
+
+int jamba_moe_timing_start(int max_launches) {
+    for (cudaEvent_t ev : g_timing.start) cudaEventDestroy(ev);
+    for (cudaEvent_t ev : g_timing.stop) cudaEventDestroy(ev);
+    g_timing.start.clear();
+    g_timing.stop.clear();
+    g_timing.kind.clear();
+    g_timing.used = 0;
+    g_timing.on = false;
+    if (max_launches <= 0) return JMOE_OK;
+    g_timing.start.resize(max_launches);
+    g_timing.stop.resize(max_launches);
+    g_timing.kind.assign(max_launches, -1);
+    for (int i = 0; i < max_launches; ++i) {
+        if (cudaEventCreate(&g_timing.start[i]) != cudaSuccess || cudaEventCreate(&g_timing.stop[i]) != cudaSuccess) {
+            g_timing.start.resize(i);
+            g_timing.stop.resize(i);
+            return JMOE_ERR_CUDA;
+        }
+    }
+    g_timing.on = true;
+    return JMOE_OK;
+}
+
+int jamba_moe_timing_collect(double* total_ms, int64_t* launches, int n_kinds) {
+    if (!total_ms || !launches || n_kinds < 0) return -JMOE_ERR_NULL;
+    const int n = n_kinds < JMOE_KERNEL_KINDS ? n_kinds : JMOE_KERNEL_KINDS;
+    for (int k = 0; k < n; ++k) {
+        total_ms[k] = 0.0;
+        launches[k] = 0;
+    }
+    for (int i = 0; i < g_timing.used; ++i) {
+        if (cudaEventSynchronize(g_timing.stop[i]) != cudaSuccess) return -JMOE_ERR_CUDA;
+        float ms = 0.0f;
+        if (cudaEventElapsedTime(&ms, g_timing.start[i], g_timing.stop[i]) != cudaSuccess) return -JMOE_ERR_CUDA;
+        const int k = g_timing.kind[i];
+        if (k >= 0 && k < n) {
+            total_ms[k] += ms;
+            launches[k] += 1;
+        }
+    }
+    return n;
+}
+
+const char* jamba_moe_kernel_name(int kind) {
+    static const char* names[JMOE_KERNEL_KINDS] = {"quantize", "router", "permute", "gather", "gemv13",
+                                                   "gemv2", "gemm13", "gemm2", "combine"};
+    return (kind >= 0 && kind < JMOE_KERNEL_KINDS) ? names[kind] : "unknown";
+}
+
+}  // extern "C"

@@ -1,0 +1,247 @@
+// Decode path of the expert FFN: few tokens per expert, so the work is bound by streaming the
+// int8 weights from HBM (Jamba rebuttal page, reply on MoE and Mamba layer interaction: MLP/MoE
+// layers are I/O bound; Jamba-1.5 paper, §3.1: the weights cross HBM -> SRAM as int8, half the
+// bytes of BF16, and are turned into BF16 right before the math).
+//
+//   gemv13: h[r][j]      = bf16( SiLU(S1[j] * (x_r . Q1[j])) * (S3[j] * (x_r . Q3[j])) )
+//   gemv2:  out[a][i]    = p_a * S2[i] * (h_r . Q2[i])        (a = the assignment of permuted row r)
+//
+// CTA = (one touched expert, 16 weight rows), 8 warps splitting K into interleaved 64-wide
+// steps.  Each lane streams 16 contiguous int8 weights of rows g and g+8 (g = lane / 4) per step
+// with 128-bit no-L1 loads, converts them exactly to bf16 in registers (bit trick, no conversion
+// unit) and feeds mma.sync m16n8k16 with the weights as A (16 rows) and up to 8*NT tokens as B.
+// Because a k-permutation applied to both operands leaves a dot product unchanged, each lane's
+// 16 consecutive k are mapped onto the fragment positions it owns, so activations are also read
+// with plain 16-byte loads (from L1/L2: they are tiny and shared by all CTAs of an expert).
+// Partial sums of the 8 warps are added in a fixed order in shared memory (deterministic), then
+// scales, SiLU * up and the routing weight are applied in fp32.
+#include "common.cuh"
+
+namespace jmoe {
+
+constexpr int kGemvWarps = 8;
+constexpr int kGemvRows = 16;
+
+struct GemvArgs {
+    const WsHeader* hdr;
+    const int32_t* perm;   // [rows] assignment index (t*K + k) of each permuted row, -1 = padding
+    const uint16_t* act;   // gemv13: x [T][d]; gemv2: h [rows][F]
+    const int8_t* qa;      // gemv13: Q1 [E][F][d]; gemv2: Q2 [E][d][F]
+    const int8_t* qb;      // gemv13: Q3 [E][F][d]; gemv2: unused
+    const float* sa;       // S1 [E][F] / S2 [E][d]
+    const float* sb;       // S3 [E][F]
+    const float* wts;      // gemv2: routing weight of each assignment [T*K]
+    uint16_t* h_out;       // gemv13: h [rows][F]
+    float* slot_out;       // gemv2: out_slot [T*K][d]
+    int64_t K;             // reduction length: d (gemv13) or F (gemv2)
+    int64_t N;             // weight rows per expert: F (gemv13) or d (gemv2)
+};
+
+template <bool kDual>
+struct WeightRegs {
+    uint4 a0, a1, b0, b1;  // rows g and g+8 of matrix a (and b)
+};
+
+template <bool kDual>
+__device__ __forceinline__ void load_weights(WeightRegs<kDual>& w, const int8_t* ra0, const int8_t* ra1,
+                                             const int8_t* rb0, const int8_t* rb1, int64_t k) {
+    w.a0 = ld_stream_v4(ra0 + k);
+    w.a1 = ld_stream_v4(ra1 + k);
+    if (kDual) {
+        w.b0 = ld_stream_v4(rb0 + k);
+        w.b1 = ld_stream_v4(rb1 + k);
+    }
+}
+
+template <int NT>
+__device__ __forceinline__ void load_acts(uint4 (&xa)[NT][2], const uint16_t* const (&rows)[NT], int64_t k) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        if (rows[nt]) {
+            xa[nt][0] = ld_nc_v4(rows[nt] + k);
+            xa[nt][1] = ld_nc_v4(rows[nt] + k + 8);
+        } else {
+            xa[nt][0] = make_uint4(0, 0, 0, 0);
+            xa[nt][1] = make_uint4(0, 0, 0, 0);
+        }
+    }
+}
+
+__device__ __forceinline__ uint32_t word(const uint4& v, int j) {
+    return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
+}
+
+template <int NT, bool kDual>
+__device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[NT][4], const WeightRegs<kDual>& w,
+                                         const uint4 (&xa)[NT][2]) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // A fragment: k positions (2c, 2c+1) <- bytes 4j, 4j+2; (2c+8, 2c+9) <- bytes 4j+1, 4j+3.
+        const uint32_t wa0 = word(w.a0, j), wa1 = word(w.a1, j);
+        const uint32_t a0 = s8x2_even_to_bf16x2(wa0), a1 = s8x2_even_to_bf16x2(wa1);
+        const uint32_t a2 = s8x2_odd_to_bf16x2(wa0), a3 = s8x2_odd_to_bf16x2(wa1);
+        uint32_t b0[NT], b1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            // activations 4j..4j+3 of this lane's 16: words 2j = (4j, 4j+1), 2j+1 = (4j+2, 4j+3)
+            const uint4& v = xa[nt][j >> 1];
+            const uint32_t lo = (j & 1) ? v.z : v.x;
+            const uint32_t hi = (j & 1) ? v.w : v.y;
+            b0[nt] = pair_lo(lo, hi);
+            b1[nt] = pair_hi(lo, hi);
+            mma_bf16_16816(acc_a[nt], a0, a1, a2, a3, b0[nt], b1[nt]);
+        }
+        if (kDual) {
+            const uint32_t wb0 = word(w.b0, j), wb1 = word(w.b1, j);
+            const uint32_t c0 = s8x2_even_to_bf16x2(wb0), c1 = s8x2_even_to_bf16x2(wb1);
+            const uint32_t c2 = s8x2_odd_to_bf16x2(wb0), c3 = s8x2_odd_to_bf16x2(wb1);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc_b[nt], c0, c1, c2, c3, b0[nt], b1[nt]);
+        }
+    }
+}
+
+// One pass over K for up to 8*NT tokens of expert e, rows [j0, j0+16).  Returns the CTA-reduced
+// accumulators in shared memory red[mat][nt][lane*4 + i] (warp 0's slice after the reduction).
+template <int NT, bool kDual>
+__device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, const uint16_t* const (&rows)[NT],
+                                          float* red /* [kGemvWarps][2][NT][128] */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, c = lane & 3;
+    const int64_t K = p.K;
+    const int8_t* ra0 = p.qa + ((int64_t)e * p.N + j0 + g) * K + 16 * c;
+    const int8_t* ra1 = ra0 + 8 * K;
+    const int8_t* rb0 = kDual ? p.qb + ((int64_t)e * p.N + j0 + g) * K + 16 * c : nullptr;
+    const int8_t* rb1 = kDual ? rb0 + 8 * K : nullptr;
+    const uint16_t* arow[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) arow[nt] = rows[nt] ? rows[nt] + 16 * c : nullptr;
+
+    float acc_a[NT][4], acc_b[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc_a[nt][i] = acc_b[nt][i] = 0.0f;
+
+    const int64_t steps = K / 64;
+    int64_t s = warp;
+    if (s < steps) {
+        WeightRegs<kDual> wn;
+        uint4 xn[NT][2];
+        load_weights<kDual>(wn, ra0, ra1, rb0, rb1, s * 64);
+        load_acts<NT>(xn, arow, s * 64);
+        for (; s < steps; s += kGemvWarps) {
+            const WeightRegs<kDual> wc = wn;
+            uint4 xc[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                xc[nt][0] = xn[nt][0];
+                xc[nt][1] = xn[nt][1];
+            }
+            if (s + kGemvWarps < steps) {  // prefetch the next step of this warp
+                load_weights<kDual>(wn, ra0, ra1, rb0, rb1, (s + kGemvWarps) * 64);
+                load_acts<NT>(xn, arow, (s + kGemvWarps) * 64);
+            }
+            mma_step<NT, kDual>(acc_a, acc_b, wc, xc);
+        }
+    }
+    // fixed-order cross-warp reduction
+    float* mine = red + (size_t)warp * 2 * NT * 128;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        *reinterpret_cast<float4*>(mine + (0 * NT + nt) * 128 + lane * 4) =
+            make_float4(acc_a[nt][0], acc_a[nt][1], acc_a[nt][2], acc_a[nt][3]);
+        if (kDual)
+            *reinterpret_cast<float4*>(mine + (1 * NT + nt) * 128 + lane * 4) =
+                make_float4(acc_b[nt][0], acc_b[nt][1], acc_b[nt][2], acc_b[nt][3]);
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < (kDual ? 2 : 1) * NT * 128; o += blockDim.x) {
+        float sum = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kGemvWarps; ++w) sum += red[(size_t)w * 2 * NT * 128 + o];
+        red[o] = sum;  // warp 0's slice now holds the totals
+    }
+    __syncthreads();
+}
+
+template <int NT, bool kDual>
+__global__ void __launch_bounds__(kGemvWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
+    __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
+    const WsHeader* hdr = p.hdr;
+    if ((int)blockIdx.y >= hdr->n_touched) return;
+    const int e = hdr->touched[blockIdx.y];
+    const int m = hdr->counts[e];
+    const int64_t row0 = hdr->seg_start[e];
+    const int64_t j0 = (int64_t)blockIdx.x * kGemvRows;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2;
+    for (int n0 = 0; n0 < m; n0 += 8 * NT) {
+        const uint16_t* rows[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int n = n0 + nt * 8 + g;
+            rows[nt] = nullptr;
+            if (n < m) {
+                if (kDual) {
+                    const int32_t a = p.perm[row0 + n];
+                    rows[nt] = p.act + (int64_t)(a / kTopK) * p.K;
+                } else {
+                    rows[nt] = p.act + (row0 + n) * p.K;
+                }
+            }
+        }
+        gemv_pass<NT, kDual>(p, e, j0, rows, red);
+        // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
+        // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
+        for (int o = threadIdx.x; o < NT * 128; o += blockDim.x) {
+            const int nt = o >> 7, l2 = (o >> 2) & 31, i = o & 3;
+            const int row = (l2 >> 2) + ((i & 2) ? 8 : 0);
+            const int n = n0 + nt * 8 + 2 * (l2 & 3) + (i & 1);
+            if (n >= m) continue;
+            const int64_t jr = j0 + row;
+            if (kDual) {
+                const float a1 = red[o] * p.sa[(int64_t)e * p.N + jr];
+                const float a3 = red[NT * 128 + o] * p.sb[(int64_t)e * p.N + jr];
+                p.h_out[(row0 + n) * p.N + jr] = f32_to_bf16_bits(silu(a1) * a3);
+            } else {
+                const int32_t a = p.perm[row0 + n];
+                p.slot_out[(int64_t)a * p.N + jr] = p.wts[a] * (p.sa[(int64_t)e * p.N + jr] * red[o]);
+            }
+        }
+        __syncthreads();  // red is reused by the next pass
+    }
+}
+
+static int gemv_nt(int64_t T) {
+    const int64_t avg = (T * kTopK + kExperts - 1) / kExperts;
+    return avg <= 6 ? 1 : (avg <= 12 ? 2 : 4);
+}
+
+template <bool kDual>
+static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st) {
+    dim3 grid((unsigned)(p.N / kGemvRows), kExperts);
+    if (nt == 1)
+        gemv_kernel<1, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
+    else if (nt == 2)
+        gemv_kernel<2, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
+    else
+        gemv_kernel<4, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
+                          const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
+                          int64_t F, cudaStream_t st) {
+    GemvArgs p{hdr, perm, x, Q1, Q3, S1, S3, nullptr, h, nullptr, d, F};
+    return launch_gemv_t<true>(p, gemv_nt(T), st);
+}
+
+cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
+                         const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
+                         cudaStream_t st) {
+    GemvArgs p{hdr, perm, h, Q2, nullptr, S2, nullptr, wts, nullptr, out_slot, F, d};
+    return launch_gemv_t<false>(p, gemv_nt(T), st);
+}
+
+}  // namespace jmoe

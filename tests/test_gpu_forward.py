@@ -1,0 +1,89 @@
+"""GPU parity of the whole layer against the fp64 oracle.
+
+y within max |y - ref| <= 2e-2 (1 + |ref|) and mean relative error <= 5e-3; routing ids exact;
+int8 codes and scales of every weight matrix bit-exact (checked while building each layer)."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+import int8_expert_weight_b200 as jm  # noqa: E402
+from gpu_layer import Layer  # noqa: E402
+from helpers import assert_routing, assert_y_close, workload  # noqa: E402
+import oracle  # noqa: E402
+
+PATHS = [pytest.param(jm.PATH_GEMV, id="gemv"), pytest.param(jm.PATH_GEMM, id="gemm")]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from int8_expert_weight_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    jm.load_library()
+
+
+def check_layer(L: Layer, path, tokens=None):
+    assert all(v == 0 for v in L.quant_mismatch.values()), L.quant_mismatch
+    y, ids, w = L.forward(path=path)
+    ref = L.oracle_forward(tokens=tokens)
+    sel = slice(None) if tokens is None else np.asarray(tokens)
+    _, _, z = oracle.route(L.x_bits[sel], L.wr, L.bias, want_logits=True)
+    assert_routing(ids[sel], w[sel], ref["ids"], ref["w"], z)
+    return assert_y_close(y[sel], ref["y"])
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    return Layer(workload("tiny"))
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_tiny_all_tokens(tiny, path):
+    check_layer(tiny, path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+@pytest.mark.parametrize("T,d,F", [(1, 256, 512), (3, 256, 512), (17, 384, 640), (129, 256, 512),
+                                   (300, 128, 128), (257, 512, 1152)])
+def test_ragged_shapes(T, d, F, path):
+    wl = dataclasses.replace(workload("tiny"), T=T, d=d, F=F)
+    check_layer(Layer(wl), path)
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_deterministic_and_status(tiny, path):
+    ws = torch.empty(jm.jamba_moe_workspace_size(tiny.wl.T, tiny.wl.d, tiny.wl.F), dtype=torch.uint8, device="cuda")
+    a = tiny.forward(path=path, workspace=ws)
+    b = tiny.forward(path=path, workspace=ws)
+    for u, v in zip(a, b):
+        assert np.array_equal(u, v)
+    assert jm.jamba_moe_read_device_status(ws) == 0
+
+
+def test_paths_agree_gemm(tiny):
+    a = tiny.forward(path=jm.PATH_GEMV)
+    b = tiny.forward(path=jm.PATH_GEMM)
+    assert np.array_equal(a[1], b[1])
+    ya = a[0].astype(np.uint32) << 16
+    yb = b[0].astype(np.uint32) << 16
+    diff = np.abs(ya.view(np.float32).astype(np.float64) - yb.view(np.float32).astype(np.float64))
+    assert diff.max() <= 2e-2
+
+
+@pytest.fixture(scope="module")
+def v01_decode():
+    return Layer(workload("v01_decode"))
+
+
+def test_v01_decode_full_size_all_tokens(v01_decode):
+    """The benchmarked workload at full size, in the benchmark's launch configuration (auto path)."""
+    check_layer(v01_decode, jm.PATH_AUTO)
+
+
+def test_v01_decode_gemm_path(v01_decode):
+    check_layer(v01_decode, jm.PATH_GEMM)
