@@ -133,6 +133,30 @@ int jamba_moe_read_device_status(const void* workspace, void* stream);
 const char* jamba_moe_status_string(int status);
 
 /*
+ * jamba_moe_forward_noalloc — jamba_moe_forward on the decode (weight-streaming) path for callers
+ * that cannot allocate device memory: code running inside a memory pool it does not own, a
+ * serving process that must not call cudaMalloc after start-up (it synchronises the device and
+ * can fail under fragmentation), or a plugin interface that only hands over inputs and outputs.
+ * The pages describe no such entry point; it has no counterpart there.
+ *
+ * Arguments are those of jamba_moe_forward without the workspace.  The scratch is one static
+ * device array of jamba_moe_noalloc_scratch_capacity() bytes (64 MiB), present on every GPU that
+ * loads this library until the process exits.  Sizes needing more
+ * (jamba_moe_noalloc_scratch_needed) return JMOE_ERR_WORKSPACE; other checks as in
+ * jamba_moe_forward.  The first call on a device looks the array's address up with that device
+ * current: make it before any stream capture.  Every call shares the array, which keeps the last
+ * call's contents (each call clears what it needs cleared); calls that may overlap on the GPU
+ * race on it.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+int jamba_moe_forward_noalloc(const uint16_t* x, const float* router_W, const float* router_bias,
+                              const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                              const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, int n_experts,
+                              int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w, void* stream);
+size_t jamba_moe_noalloc_scratch_capacity(void);
+/* Scratch bytes jamba_moe_forward_noalloc needs for these sizes (0 = unsupported sizes). */
+size_t jamba_moe_noalloc_scratch_needed(int64_t T, int64_t d, int64_t ffn);
+
+/*
  * Kernel timing (for the benchmark's roofline figures).
  * jamba_moe_timing_start(max_launches) makes every following launch of this library record a
  * pair of CUDA events on its stream, until max_launches pairs are recorded, and forgets any

@@ -59,6 +59,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_timing_start.argtypes = [c_int]
     lib.jamba_moe_timing_collect.restype = c_int
     lib.jamba_moe_timing_collect.argtypes = [vp, vp, c_int]
+    lib.jamba_moe_forward_noalloc.restype = c_int
+    lib.jamba_moe_forward_noalloc.argtypes = fwd_args[:17] + [vp]
+    lib.jamba_moe_noalloc_scratch_capacity.restype = sz
+    lib.jamba_moe_noalloc_scratch_capacity.argtypes = []
+    lib.jamba_moe_noalloc_scratch_needed.restype = sz
+    lib.jamba_moe_noalloc_scratch_needed.argtypes = [i64, i64, i64]
     lib.jamba_moe_kernel_name.restype = ctypes.c_char_p
     lib.jamba_moe_kernel_name.argtypes = [c_int]
     _lib = lib
@@ -168,6 +174,31 @@ def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Opti
                                     workspace.data_ptr(), workspace.numel(), _stream_ptr(stream), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward")
+    return y, topk_ids, topk_w
+
+
+def jamba_moe_forward_noalloc(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor],
+                              Q1: torch.Tensor, S1: torch.Tensor, Q3: torch.Tensor, S3: torch.Tensor,
+                              Q2: torch.Tensor, S2: torch.Tensor, y: torch.Tensor, topk_ids: torch.Tensor,
+                              topk_w: torch.Tensor, stream: Optional[torch.cuda.Stream] = None):
+    """jamba_moe_forward without a workspace, for callers that cannot allocate device memory: the
+    scratch is the library's static 64 MiB device array.  All outputs are caller-provided, so
+    this wrapper allocates nothing either.  Calls that overlap on the GPU race on the array."""
+    lib = load_library()
+    T, d = x.shape
+    E, ffn = Q1.shape[0], Q1.shape[1]
+    for t, n, dt in ((x, "x", torch.bfloat16), (y, "y", torch.bfloat16), (router_W, "router_W", torch.float32),
+                     (Q1, "Q1", torch.int8), (Q3, "Q3", torch.int8), (Q2, "Q2", torch.int8),
+                     (S1, "S1", torch.float32), (S3, "S3", torch.float32), (S2, "S2", torch.float32),
+                     (topk_ids, "topk_ids", torch.int32), (topk_w, "topk_w", torch.float32)):
+        _check(t, n, dt)
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    st = lib.jamba_moe_forward_noalloc(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
+                                       S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
+                                       T, d, ffn, E, TOP_K, y.data_ptr(), topk_ids.data_ptr(), topk_w.data_ptr(),
+                                       _stream_ptr(stream))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_forward_noalloc")
     return y, topk_ids, topk_w
 
 
