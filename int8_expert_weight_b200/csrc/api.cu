@@ -21,11 +21,17 @@ cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_
                          const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
                          cudaStream_t st);
 cudaError_t launch_combine(const float* slots, int64_t T, int64_t d, uint16_t* y, cudaStream_t st, int num_sms);
+cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const int8_t* Q1,
+                          const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
+                          int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2, const float* S2,
+                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st);
 
 namespace {
 
 constexpr int64_t kMaxT = int64_t(1) << 20;
 constexpr int64_t kMaxDim = 32768;
+constexpr int64_t kGemvMaxTokens = 128;  // auto path: GEMV up to 2*128/16 = 16 rows per expert on average
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -156,11 +162,10 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
     uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
     uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
     float* slots = reinterpret_cast<float*>(ws + L.slots);
-    (void)x_perm;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = num_sms_current();
-    if (path == JMOE_PATH_AUTO) path = JMOE_PATH_GEMV;
-    if (path == JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;  // grouped tensor-core path not built yet
+    // Few tokens per expert: stream the weights (GEMV); otherwise grouped tensor-core GEMMs.
+    if (path == JMOE_PATH_AUTO) path = (T <= kGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
 
     cudaError_t e;
     {
@@ -173,16 +178,34 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
         e = launch_permute(ids, T, hdr, perm, inv, st);
     }
     if (e != cudaSuccess) return JMOE_ERR_CUDA;
-    {
-        TimedLaunch t(JMOE_KERNEL_GEMV13, st);
-        e = launch_gemv13(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st);
+    if (path == JMOE_PATH_GEMV) {
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV13, st);
+            e = launch_gemv13(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV2, st);
+            e = launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    } else {
+        {
+            TimedLaunch t(JMOE_KERNEL_GATHER, st);
+            e = launch_gather(x, perm, hdr, d, L.rows_cap, x_perm, st, sms);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMM13, st);
+            e = launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMM2, st);
+            e = launch_gemm2(hdr, perm, h, Q2, S2, wts, slots, L.rows_cap, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
     }
-    if (e != cudaSuccess) return JMOE_ERR_CUDA;
-    {
-        TimedLaunch t(JMOE_KERNEL_GEMV2, st);
-        e = launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st);
-    }
-    if (e != cudaSuccess) return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_COMBINE, st);
         e = launch_combine(slots, T, d, y, st, sms);

@@ -1,0 +1,389 @@
+// Prefill path of the expert FFN: grouped GEMMs on the 5th-generation tensor cores (tcgen05), with
+// the ExpertsInt8 dequantization inside the kernel (Jamba-1.5 paper, §3.1: int8 weight tiles move
+// HBM -> SRAM and are turned into BF16 there, right before the matrix math).
+//
+//   gemm13: h[r][j] = bf16( SiLU(S1[j] * (x_r . Q1[j])) * (S3[j] * (x_r . Q3[j])) )   tile: 128 rows x
+//           (128 j of Q1 | the same 128 j of Q3), so both halves of SwiGLU meet in one accumulator
+//   gemm2:  out[a][i] = p_a * S2[i] * (h_r . Q2[i])                                   tile: 128 rows x BN i
+//
+// One CTA per output tile, 192 threads:
+//   warp 0      TMA producer: activation tile (bf16, SWIZZLE_128B) + int8 weight tile per 64-wide K step
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16, fp32 in TMEM
+//   warps 2-5   converters: int8 tile -> bf16 in the canonical SWIZZLE_128B K-major layout, then the
+//               epilogue (tcgen05.ld, scales, SiLU * up or routing weight, stores)
+// A 3-stage ring of (activations, int8 weights, bf16 weights) buffers; full / converted / empty
+// mbarriers per stage.  Every wait is bounded: on timeout the kernel records JMOE_DEV_TIMEOUT in the
+// workspace status word, the other roles stop at their next wait, outstanding copies and MMAs are
+// waited for (bounded), TMEM is released and the CTA returns.
+//
+// Tiles are ordered expert by expert; inside an expert, bands of M tiles keep their activations
+// resident in L2 while every N tile of the weights streams past once per band.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "tc.cuh"
+
+namespace jmoe {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kStages = 3;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kMaxPolls = 1u << 22;
+
+struct GemmArgs {
+    WsHeader* hdr;
+    const int32_t* perm;  // assignment index of each permuted row, -1 = padding
+    const float* sa;      // gemm13: S1 [E][N]; gemm2: S2 [E][N]
+    const float* sb;      // gemm13: S3 [E][N]
+    const float* wts;     // gemm2: routing weight per assignment
+    uint16_t* h_out;      // gemm13: h [rows][N]
+    float* slot_out;      // gemm2: out_slot [T*K][N]
+    int K;                // d (gemm13) or ffn (gemm2)
+    int N;                // weight rows per expert and matrix: ffn (gemm13) or d (gemm2)
+    int n_tiles;          // N tiles per M tile
+    int band;             // M tiles per raster band
+};
+
+template <int BN>
+struct StageLayout {
+    static constexpr int kA = kBM * kBK * 2;   // bf16 activations
+    static constexpr int kBbf = BN * kBK * 2;  // bf16 weights (converted)
+    static constexpr int kBq = BN * kBK;       // int8 weights (as loaded)
+    static constexpr int kStage = kA + kBbf + kBq;
+    static constexpr int kBars = 8 * (3 * kStages + 1);
+    static constexpr int kSmem = kStages * kStage + 1024 + 256;
+};
+
+// bf16x2 of bytes (i0, i1) of w, exactly: (0x4300 | low7) - (0x4300 | sign bit), in k order.
+__device__ __forceinline__ uint32_t s8pair_to_bf16x2(uint32_t lo7, uint32_t hi1, uint32_t sel) {
+    const uint32_t v = __byte_perm(lo7, 0x43434343u, sel);
+    const uint32_t c = __byte_perm(hi1, 0x43434343u, sel);
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(c));
+    return r;
+}
+
+__device__ __forceinline__ void convert16(const uint4 v, uint32_t (&o)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo7 = w[i] & 0x7F7F7F7Fu, hi1 = w[i] & 0x80808080u;
+        o[2 * i] = s8pair_to_bf16x2(lo7, hi1, 0x4140);      // bytes 0, 1
+        o[2 * i + 1] = s8pair_to_bf16x2(lo7, hi1, 0x4342);  // bytes 2, 3
+    }
+}
+
+__device__ __forceinline__ void fail(WsHeader* hdr, volatile int* abort) {
+    *abort = 1;
+    set_status(hdr, JMOE_DEV_TIMEOUT);
+}
+
+template <bool kDual, int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmB1, GemmArgs p) {
+    using SL = StageLayout<BN>;
+    static_assert(!kDual || BN == 256, "the SwiGLU tile pairs 128 gate rows with 128 up rows");
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint32_t tmem_holder;
+    __shared__ volatile int abort_flag;
+
+    // ---- which tile: expert, then band of M tiles, then N tile, then M tile within the band
+    const WsHeader* hdr = p.hdr;
+    int L = blockIdx.x, e = -1, base = 0, mt_e = 0;
+    for (int i = 0; i < kExperts; ++i) {
+        const int mt = hdr->tile_start[i + 1] - hdr->tile_start[i];
+        if (L < base + mt * p.n_tiles) {
+            e = i;
+            mt_e = mt;
+            break;
+        }
+        base += mt * p.n_tiles;
+    }
+    if (e < 0) return;  // past the real tiles: nothing was taken yet
+    const int local = L - base;
+    const int band = local / (p.band * p.n_tiles);
+    const int m_first = band * p.band;
+    const int bsz = min(p.band, mt_e - m_first);
+    const int within = local - band * p.band * p.n_tiles;
+    const int n_tile = within / bsz;
+    const int m_tile = m_first + within % bsz;
+    const int a_row0 = hdr->seg_start[e] + m_tile * kBM;
+    const int w_row0 = e * p.N + n_tile * (kDual ? BN / 2 : BN);
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * SL::kStage);
+    uint64_t* full_tma = bars;
+    uint64_t* full_bf = bars + kStages;
+    uint64_t* empty = bars + 2 * kStages;
+    uint64_t* acc_full = bars + 3 * kStages;
+    auto sA = [&](int s) { return smem + s * SL::kStage; };
+    auto sBbf = [&](int s) { return smem + s * SL::kStage + SL::kA; };
+    auto sBq = [&](int s) { return smem + s * SL::kStage + SL::kA + SL::kBbf; };
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            tc::mbar_init(&full_tma[s], 1);
+            tc::mbar_init(&full_bf[s], 32 * 4);
+            tc::mbar_init(&empty[s], 1);
+        }
+        tc::mbar_init(acc_full, 1);
+        abort_flag = 0;
+        tc::mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tc::prefetch_tmap(&tmA);
+        tc::prefetch_tmap(&tmB0);
+        if (kDual) tc::prefetch_tmap(&tmB1);
+    }
+    if (warp == 1) tc::tmem_alloc(&tmem_holder, BN);
+    tc::tc_fence_before();
+    __syncthreads();
+    tc::tc_fence_after();
+    const uint32_t tmem = tmem_holder;
+    const int KB = p.K / kBK;
+    constexpr uint32_t kTxBytes = SL::kA + SL::kBq;
+    constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, BN);
+    int issued_round[kStages] = {-1, -1, -1};  // producer: last round issued on each stage
+    int mma_issued = 0;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % kStages, r = kb / kStages;
+                if (r > 0 && !tc::mbar_wait_bounded(&empty[s], (r - 1) & 1, &abort_flag, kMaxPolls)) {
+                    if (!abort_flag) fail(p.hdr, &abort_flag);
+                    break;
+                }
+                tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
+                tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
+                if (kDual) {
+                    tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                    tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                } else {
+                    tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                }
+                issued_round[s] = r;
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int kb = 0; kb < KB; ++kb) {
+                const int s = kb % kStages, r = kb / kStages;
+                if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls) ||
+                    !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, kMaxPolls)) {
+                    if (!abort_flag) fail(p.hdr, &abort_flag);
+                    break;
+                }
+                tc::tc_fence_after();
+                const uint64_t adesc = tc::sw128_kmajor_desc(tc::smem_u32(sA(s)));
+                const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sBbf(s)));
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per 16-element K step = +2 in the address field
+                    tc::mma_bf16_ss(tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+                tc::mma_commit(&empty[s]);
+                ++mma_issued;
+            }
+            tc::mma_commit(acc_full);  // arrives once every MMA issued above has completed
+        }
+        __syncwarp();
+    } else {
+        // ---- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte chunk c of row r
+        // stored at chunk c ^ (r & 7) of the row's 128 bytes)
+        const int t = threadIdx.x - 64;
+        for (int kb = 0; kb < KB; ++kb) {
+            const int s = kb % kStages, r = kb / kStages;
+            if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls)) {
+                if (!abort_flag) fail(p.hdr, &abort_flag);
+                break;
+            }
+            const uint8_t* q8 = sBq(s);
+            uint8_t* bf = sBbf(s);
+#pragma unroll
+            for (int i = 0; i < BN * 4 / 128; ++i) {
+                const int qi = t + 128 * i, row = qi >> 2, c = qi & 3;
+                const uint4 v = *reinterpret_cast<const uint4*>(q8 + row * kBK + c * 16);
+                uint32_t o[8];
+                convert16(v, o);
+                uint8_t* rp = bf + row * 128;
+                *reinterpret_cast<uint4*>(rp + (((2 * c) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(rp + (((2 * c + 1) ^ (row & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+            tc::fence_proxy_async_smem();
+            tc::mbar_arrive(&full_bf[s]);
+        }
+        // ---- epilogue
+        bool ok = tc::mbar_wait_bounded(acc_full, 0, &abort_flag, kMaxPolls);
+        if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
+        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+        tc::tc_fence_after();
+        if (ok) {
+            const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 are this warp's
+            const int row = q * 32 + lane;
+            const int64_t gr = (int64_t)a_row0 + row;
+            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+            if (kDual) {
+                const int j0 = n_tile * (BN / 2);
+                const float* s1 = p.sa + (int64_t)e * p.N + j0;
+                const float* s3 = p.sb + (int64_t)e * p.N + j0;
+                uint16_t* hrow = p.h_out + gr * p.N + j0;
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    uint32_t a1[32], a3[32];
+                    tc::tmem_ld32(tbase + c, a1);
+                    tc::tmem_ld32(tbase + BN / 2 + c, a3);
+                    tc::tmem_wait_ld();
+                    uint32_t packed[16];
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const float g0 = __uint_as_float(a1[i]) * __ldg(s1 + c + i);
+                        const float g1 = __uint_as_float(a1[i + 1]) * __ldg(s1 + c + i + 1);
+                        const float u0 = __uint_as_float(a3[i]) * __ldg(s3 + c + i);
+                        const float u1 = __uint_as_float(a3[i + 1]) * __ldg(s3 + c + i + 1);
+                        packed[i / 2] = (uint32_t)f32_to_bf16_bits(silu(g0) * u0) |
+                                        ((uint32_t)f32_to_bf16_bits(silu(g1) * u1) << 16);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(hrow + c);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                }
+            } else {
+                const int i0 = n_tile * BN;
+                const int32_t a = p.perm[gr];
+                const float wt = a >= 0 ? p.wts[a] : 0.0f;
+                const float* s2 = p.sa + (int64_t)e * p.N + i0;
+                float* orow = p.slot_out + (int64_t)(a >= 0 ? a : 0) * p.N + i0;
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v[32];
+                    tc::tmem_ld32(tbase + c, v);
+                    tc::tmem_wait_ld();
+                    if (a >= 0) {
+                        float4* dst = reinterpret_cast<float4*>(orow + c);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            float4 o;
+                            o.x = wt * (__ldg(s2 + c + 4 * k + 0) * __uint_as_float(v[4 * k + 0]));
+                            o.y = wt * (__ldg(s2 + c + 4 * k + 1) * __uint_as_float(v[4 * k + 1]));
+                            o.z = wt * (__ldg(s2 + c + 4 * k + 2) * __uint_as_float(v[4 * k + 2]));
+                            o.w = wt * (__ldg(s2 + c + 4 * k + 3) * __uint_as_float(v[4 * k + 3]));
+                            dst[k] = o;
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    // ---- teardown: after an abort, let in-flight copies and MMAs finish (bounded) before TMEM goes
+    tc::tc_fence_before();
+    __syncthreads();
+    if (abort_flag) {
+        if (warp == 0 && lane == 0) {
+            for (int s = 0; s < kStages; ++s) {
+                if (issued_round[s] < 0) continue;
+                // a copy of round r completes phase r of full_tma[s]; waiting ignores the abort flag
+                for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(&full_tma[s], issued_round[s] & 1); ++i)
+                    __nanosleep(64);
+            }
+        }
+        if (warp == 1 && lane == 0 && mma_issued > 0) {
+            for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(acc_full, 0); ++i) __nanosleep(64);
+        }
+        __syncthreads();
+    }
+    if (warp == 1) {
+        tc::tc_fence_after();
+        tc::tmem_dealloc(tmem, BN);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// 2D row-major [rows][cols] tensor, box [box_rows][box_cols].
+bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_bytes, uint64_t rows, uint64_t cols,
+              uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int band_for(int K) {
+    // keep a band's activation tiles (band * 128 rows * K * 2 bytes) near 24 MB of L2
+    const int64_t per_tile = (int64_t)kBM * K * 2;
+    int b = (int)((24ll << 20) / per_tile);
+    return b < 1 ? 1 : (b > 16 ? 16 : b);
+}
+
+template <bool kDual, int BN>
+cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const GemmArgs& p,
+                          int64_t m_tiles_cap, cudaStream_t st) {
+    using SL = StageLayout<BN>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SL::kSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = m_tiles_cap * p.n_tiles;
+    gemm_tc_kernel<kDual, BN><<<(unsigned)grid, kGemmThreads, SL::kSmem, st>>>(ta, tb0, tb1, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// h = SwiGLU(x_perm . Q1^T, x_perm . Q3^T) per expert segment; rows_cap = permuted-row capacity.
+cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const int8_t* Q1,
+                          const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
+                          int64_t d, int64_t F, cudaStream_t st) {
+    CUtensorMap ta, tb0, tb1;
+    if (!make_map(&ta, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kBM, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr, perm, S1, S3, nullptr, h, nullptr, (int)d, (int)F, (int)(F / 128), band_for((int)d)};
+    return launch_gemm_t<true, 256>(ta, tb0, tb1, p, rows_cap / kBM, st);
+}
+
+// out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment.
+cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2, const float* S2,
+                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st) {
+    const int BN = (d % 256 == 0) ? 256 : 128;
+    CUtensorMap ta, tb0;
+    if (!make_map(&ta, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * d, F, BN, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr, perm, S2, nullptr, wts, nullptr, out_slot, (int)F, (int)d, (int)(d / BN), band_for((int)F)};
+    if (BN == 256) return launch_gemm_t<false, 256>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    return launch_gemm_t<false, 128>(ta, tb0, tb0, p, rows_cap / kBM, st);
+}
+
+}  // namespace jmoe

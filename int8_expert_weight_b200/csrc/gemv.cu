@@ -42,31 +42,6 @@ struct WeightRegs {
     uint4 a0, a1, b0, b1;  // rows g and g+8 of matrix a (and b)
 };
 
-template <bool kDual>
-__device__ __forceinline__ void load_weights(WeightRegs<kDual>& w, const int8_t* ra0, const int8_t* ra1,
-                                             const int8_t* rb0, const int8_t* rb1, int64_t k) {
-    w.a0 = ld_stream_v4(ra0 + k);
-    w.a1 = ld_stream_v4(ra1 + k);
-    if (kDual) {
-        w.b0 = ld_stream_v4(rb0 + k);
-        w.b1 = ld_stream_v4(rb1 + k);
-    }
-}
-
-template <int NT>
-__device__ __forceinline__ void load_acts(uint4 (&xa)[NT][2], const uint16_t* const (&rows)[NT], int64_t k) {
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-        if (rows[nt]) {
-            xa[nt][0] = ld_nc_v4(rows[nt] + k);
-            xa[nt][1] = ld_nc_v4(rows[nt] + k + 8);
-        } else {
-            xa[nt][0] = make_uint4(0, 0, 0, 0);
-            xa[nt][1] = make_uint4(0, 0, 0, 0);
-        }
-    }
-}
-
 __device__ __forceinline__ uint32_t word(const uint4& v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
@@ -101,21 +76,26 @@ __device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[N
     }
 }
 
-// One pass over K for up to 8*NT tokens of expert e, rows [j0, j0+16).  Returns the CTA-reduced
-// accumulators in shared memory red[mat][nt][lane*4 + i] (warp 0's slice after the reduction).
-template <int NT, bool kDual>
+// One pass over K for up to 8*NT tokens of expert e, rows [j0, j0+16).  Warp w takes the k-steps
+// w, w+8, w+16, ...; U consecutive steps of a warp are loaded into separate registers before any is
+// consumed, so each lane keeps U*(2 or 4)*16 bytes of weights in flight.  Addresses advance by one
+// pointer increment per batch; the U steps are immediate offsets from it.  Rows of tokens past the
+// expert's count point at a valid row: their MMA columns are computed and then ignored.
+// Returns the CTA-reduced accumulators in shared memory red[mat][nt][lane*4 + i].
+template <int NT, bool kDual, int U>
 __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, const uint16_t* const (&rows)[NT],
                                           float* red /* [kGemvWarps][2][NT][128] */) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int64_t K = p.K;
-    const int8_t* ra0 = p.qa + ((int64_t)e * p.N + j0 + g) * K + 16 * c;
-    const int8_t* ra1 = ra0 + 8 * K;
-    const int8_t* rb0 = kDual ? p.qb + ((int64_t)e * p.N + j0 + g) * K + 16 * c : nullptr;
-    const int8_t* rb1 = kDual ? rb0 + 8 * K : nullptr;
-    const uint16_t* arow[NT];
+    constexpr int kStride = kGemvWarps * 64;  // bytes (int8) / elements (bf16) between a warp's steps
+    const int8_t* pa0 = p.qa + ((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64;
+    const int8_t* pa1 = pa0 + 8 * K;
+    const int8_t* pb0 = kDual ? p.qb + ((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64 : nullptr;
+    const int8_t* pb1 = kDual ? pb0 + 8 * K : nullptr;
+    const uint16_t* px[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) arow[nt] = rows[nt] ? rows[nt] + 16 * c : nullptr;
+    for (int nt = 0; nt < NT; ++nt) px[nt] = rows[nt] + 16 * c + warp * 64;
 
     float acc_a[NT][4], acc_b[NT][4];
 #pragma unroll
@@ -123,27 +103,37 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc_a[nt][i] = acc_b[nt][i] = 0.0f;
 
-    const int64_t steps = K / 64;
-    int64_t s = warp;
-    if (s < steps) {
-        WeightRegs<kDual> wn;
-        uint4 xn[NT][2];
-        load_weights<kDual>(wn, ra0, ra1, rb0, rb1, s * 64);
-        load_acts<NT>(xn, arow, s * 64);
-        for (; s < steps; s += kGemvWarps) {
-            const WeightRegs<kDual> wc = wn;
-            uint4 xc[NT][2];
+    const int steps = (int)(K / 64);
+    for (int s0 = warp; s0 < steps; s0 += kGemvWarps * U) {
+        WeightRegs<kDual> w[U];
+        uint4 xa[U][NT][2];
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                xc[nt][0] = xn[nt][0];
-                xc[nt][1] = xn[nt][1];
+        for (int u = 0; u < U; ++u) {
+            if (s0 + u * kGemvWarps < steps) {
+                w[u].a0 = ld_stream_v4(pa0 + u * kStride);
+                w[u].a1 = ld_stream_v4(pa1 + u * kStride);
+                if (kDual) {
+                    w[u].b0 = ld_stream_v4(pb0 + u * kStride);
+                    w[u].b1 = ld_stream_v4(pb1 + u * kStride);
+                }
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    xa[u][nt][0] = ld_nc_v4(px[nt] + u * kStride);
+                    xa[u][nt][1] = ld_nc_v4(px[nt] + u * kStride + 8);
+                }
             }
-            if (s + kGemvWarps < steps) {  // prefetch the next step of this warp
-                load_weights<kDual>(wn, ra0, ra1, rb0, rb1, (s + kGemvWarps) * 64);
-                load_acts<NT>(xn, arow, (s + kGemvWarps) * 64);
-            }
-            mma_step<NT, kDual>(acc_a, acc_b, wc, xc);
         }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+            if (s0 + u * kGemvWarps < steps) mma_step<NT, kDual>(acc_a, acc_b, w[u], xa[u]);
+        pa0 += U * kStride;
+        pa1 += U * kStride;
+        if (kDual) {
+            pb0 += U * kStride;
+            pb1 += U * kStride;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) px[nt] += U * kStride;
     }
     // fixed-order cross-warp reduction
     float* mine = red + (size_t)warp * 2 * NT * 128;
@@ -181,17 +171,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kerne
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
             const int n = n0 + nt * 8 + g;
-            rows[nt] = nullptr;
-            if (n < m) {
-                if (kDual) {
-                    const int32_t a = p.perm[row0 + n];
-                    rows[nt] = p.act + (int64_t)(a / kTopK) * p.K;
-                } else {
-                    rows[nt] = p.act + (row0 + n) * p.K;
-                }
+            const int nn = n < m ? n : 0;  // past the count: any valid row, its column is ignored
+            if (kDual) {
+                const int32_t a = p.perm[row0 + nn];
+                rows[nt] = p.act + (int64_t)(a / kTopK) * p.K;
+            } else {
+                rows[nt] = p.act + (row0 + nn) * p.K;
             }
         }
-        gemv_pass<NT, kDual>(p, e, j0, rows, red);
+        gemv_pass<NT, kDual, (kDual ? 2 : 4)>(p, e, j0, rows, red);
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
         for (int o = threadIdx.x; o < NT * 128; o += blockDim.x) {

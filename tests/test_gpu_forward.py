@@ -87,3 +87,53 @@ def test_v01_decode_full_size_all_tokens(v01_decode):
 
 def test_v01_decode_gemm_path(v01_decode):
     check_layer(v01_decode, jm.PATH_GEMM)
+
+
+def sample_tokens(ids_ref: np.ndarray, n_strided: int) -> np.ndarray:
+    """Evenly strided tokens plus, for every expert, the first and last token routed to it (the first
+    and last rows of its permuted segment, since the permutation keeps token order)."""
+    T = ids_ref.shape[0]
+    toks = set(np.linspace(0, T - 1, n_strided).round().astype(int).tolist())
+    for e in range(16):
+        hit = np.nonzero((ids_ref == e).any(1))[0]
+        if hit.size:
+            toks.update([int(hit[0]), int(hit[-1]), int(hit[hit.size // 2])])
+    return np.array(sorted(toks), dtype=np.int64)
+
+
+def check_sampled(L: Layer, path, n_strided):
+    assert all(v == 0 for v in L.quant_mismatch.values()), L.quant_mismatch
+    y, ids, w = L.forward(path=path)
+    ids_o, w_o, z = oracle.route(L.x_bits, L.wr, L.bias, want_logits=True)
+    assert_routing(ids, w, ids_o, w_o, z)  # every token
+    toks = sample_tokens(ids_o, n_strided)
+    ref = L.oracle_forward(tokens=toks)
+    return assert_y_close(y[toks], ref["y"], f"y on {toks.size} sampled tokens")
+
+
+@pytest.fixture(scope="module")
+def v01_prefill():
+    return Layer(workload("v01_prefill"))
+
+
+def test_v01_prefill_sampled(v01_prefill):
+    check_sampled(v01_prefill, jm.PATH_AUTO, 256)
+
+
+def test_skewed_sampled():
+    check_sampled(Layer(workload("skewed")), jm.PATH_AUTO, 256)
+
+
+@pytest.mark.slow
+def test_large_prefill_sampled():
+    check_sampled(Layer(workload("large_prefill")), jm.PATH_AUTO, 96)
+
+
+@pytest.mark.slow
+def test_large_decode_all_paths():
+    L = Layer(workload("large_decode"))
+    toks = np.arange(0, 64, 4)
+    for path in (jm.PATH_AUTO, jm.PATH_GEMM):
+        y, ids, w = L.forward(path=path)
+        ref = L.oracle_forward(tokens=toks)
+        assert_y_close(y[toks], ref["y"], f"large decode path {path}")
