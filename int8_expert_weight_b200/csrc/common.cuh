@@ -51,14 +51,18 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 // ------------------------------------------------------------------ int8 -> bf16, exact
 // For a byte b (two's complement q), the bf16 with exponent 0x86 and mantissa b & 0x7F is
 // 128 + (b & 0x7F); subtracting 128 (b >= 0) or 256 (b < 0) leaves exactly q.  Both bf16
-// operands and the integer result (|q| <= 128) are exact, so the subtraction is exact.
-// Works on bytes 0 and 2 of a 32-bit word, giving a bf16x2 (byte 0 in the low half).
+// operands and the integer result (|q| <= 128) are exact, so the subtraction is exact.  It is
+// done as one bf16x2 fma, c * (-1) + v.
+__device__ __forceinline__ uint32_t bf16x2_v_minus_c(uint32_t v, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(c), "r"(0xBF80BF80u), "r"(v));
+    return r;
+}
+// Bytes 0 and 2 of a 32-bit word as a bf16x2 (byte 0 in the low half).
 __device__ __forceinline__ uint32_t s8x2_even_to_bf16x2(uint32_t w) {
     const uint32_t v = (w & 0x007F007Fu) | 0x43004300u;
     const uint32_t c = (w & 0x00800080u) | 0x43004300u;
-    uint32_t r;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(c));
-    return r;
+    return bf16x2_v_minus_c(v, c);
 }
 // Bytes 1 and 3 of the word.
 __device__ __forceinline__ uint32_t s8x2_odd_to_bf16x2(uint32_t w) { return s8x2_even_to_bf16x2(w >> 8); }

@@ -6,15 +6,16 @@
 //           (128 j of Q1 | the same 128 j of Q3), so both halves of SwiGLU meet in one accumulator
 //   gemm2:  out[a][i] = p_a * S2[i] * (h_r . Q2[i])                                   tile: 128 rows x BN i
 //
-// One CTA per output tile, 192 threads:
-//   warp 0      TMA producer: activation tile (bf16, SWIZZLE_128B) + int8 weight tile per 64-wide K step
-//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16, fp32 in TMEM
-//   warps 2-5   converters: int8 tile -> bf16 in the canonical SWIZZLE_128B K-major layout, then the
-//               epilogue (tcgen05.ld, scales, SiLU * up or routing weight, stores)
-// A 3-stage ring of (activations, int8 weights, bf16 weights) buffers; full / converted / empty
-// mbarriers per stage.  Every wait is bounded: on timeout the kernel records JMOE_DEV_TIMEOUT in the
-// workspace status word, the other roles stop at their next wait, outstanding copies and MMAs are
-// waited for (bounded), TMEM is released and the CTA returns.
+// Persistent: one CTA per SM walks the tile list with stride gridDim.x; 448 threads in roles:
+//   warp 0       TMA producer: activation tile (bf16, SWIZZLE_128B) + int8 weight tile per 64-wide K step
+//   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16, fp32 in TMEM
+//   warps 2-9    converters: int8 tile -> bf16 in the canonical SWIZZLE_128B K-major layout
+//   warps 10-13  epilogue: tcgen05.ld, scales, SiLU * up or routing weight, global stores
+// A 3-stage ring of (activations, int8 weights, bf16 weights) buffers with full / converted / empty
+// mbarriers, and two TMEM accumulators (full / empty mbarriers) so that a tile's epilogue overlaps
+// the next tile's main loop.  Every wait is bounded: on timeout the kernel records
+// JMOE_DEV_TIMEOUT in the workspace status word, the other roles stop at their next wait,
+// outstanding copies and MMAs are waited for (bounded), TMEM is released and the CTA returns.
 //
 // Tiles are ordered expert by expert; inside an expert, bands of M tiles keep their activations
 // resident in L2 while every N tile of the weights streams past once per band.
@@ -28,7 +29,9 @@ namespace jmoe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kStages = 3;
-constexpr int kGemmThreads = 192;
+constexpr int kConvWarps = 8;
+constexpr int kEpiWarps = 4;
+constexpr int kGemmThreads = (2 + kConvWarps + kEpiWarps) * 32;
 constexpr uint32_t kMaxPolls = 1u << 22;
 
 struct GemmArgs {
@@ -51,17 +54,12 @@ struct StageLayout {
     static constexpr int kBbf = BN * kBK * 2;  // bf16 weights (converted)
     static constexpr int kBq = BN * kBK;       // int8 weights (as loaded)
     static constexpr int kStage = kA + kBbf + kBq;
-    static constexpr int kBars = 8 * (3 * kStages + 1);
     static constexpr int kSmem = kStages * kStage + 1024 + 256;
 };
 
-// bf16x2 of bytes (i0, i1) of w, exactly: (0x4300 | low7) - (0x4300 | sign bit), in k order.
+// bf16x2 of two bytes of w, exactly, in k order: (0x4300 | low 7 bits) - (0x4300 | sign bit).
 __device__ __forceinline__ uint32_t s8pair_to_bf16x2(uint32_t lo7, uint32_t hi1, uint32_t sel) {
-    const uint32_t v = __byte_perm(lo7, 0x43434343u, sel);
-    const uint32_t c = __byte_perm(hi1, 0x43434343u, sel);
-    uint32_t r;
-    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(c));
-    return r;
+    return bf16x2_v_minus_c(__byte_perm(lo7, 0x43434343u, sel), __byte_perm(hi1, 0x43434343u, sel));
 }
 
 __device__ __forceinline__ void convert16(const uint4 v, uint32_t (&o)[8]) {
@@ -79,45 +77,55 @@ __device__ __forceinline__ void fail(WsHeader* hdr, volatile int* abort) {
     set_status(hdr, JMOE_DEV_TIMEOUT);
 }
 
+struct TileCoord {
+    int e, m_tile, n_tile;
+};
+
+// Tile L of the list: expert by expert; inside an expert, bands of `band` M tiles, N tiles of a
+// band in order, M tiles of the band fastest.  Returns false past the last tile.
+__device__ __forceinline__ bool tile_coord(const WsHeader* hdr, const GemmArgs& p, int L, TileCoord& t) {
+    int base = 0;
+    for (int i = 0; i < kExperts; ++i) {
+        const int mt = hdr->tile_start[i + 1] - hdr->tile_start[i];
+        if (L < base + mt * p.n_tiles) {
+            const int local = L - base;
+            const int band = local / (p.band * p.n_tiles);
+            const int m_first = band * p.band;
+            const int bsz = min(p.band, mt - m_first);
+            const int within = local - band * p.band * p.n_tiles;
+            t.e = i;
+            t.n_tile = within / bsz;
+            t.m_tile = m_first + within % bsz;
+            return true;
+        }
+        base += mt * p.n_tiles;
+    }
+    return false;
+}
+
 template <bool kDual, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, GemmArgs p) {
     using SL = StageLayout<BN>;
     static_assert(!kDual || BN == 256, "the SwiGLU tile pairs 128 gate rows with 128 up rows");
+    constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
 
-    // ---- which tile: expert, then band of M tiles, then N tile, then M tile within the band
     const WsHeader* hdr = p.hdr;
-    int L = blockIdx.x, e = -1, base = 0, mt_e = 0;
-    for (int i = 0; i < kExperts; ++i) {
-        const int mt = hdr->tile_start[i + 1] - hdr->tile_start[i];
-        if (L < base + mt * p.n_tiles) {
-            e = i;
-            mt_e = mt;
-            break;
-        }
-        base += mt * p.n_tiles;
-    }
-    if (e < 0) return;  // past the real tiles: nothing was taken yet
-    const int local = L - base;
-    const int band = local / (p.band * p.n_tiles);
-    const int m_first = band * p.band;
-    const int bsz = min(p.band, mt_e - m_first);
-    const int within = local - band * p.band * p.n_tiles;
-    const int n_tile = within / bsz;
-    const int m_tile = m_first + within % bsz;
-    const int a_row0 = hdr->seg_start[e] + m_tile * kBM;
-    const int w_row0 = e * p.N + n_tile * (kDual ? BN / 2 : BN);
+    const int total = hdr->tile_start[kExperts] * p.n_tiles;
+    if ((int)blockIdx.x >= total) return;  // no tile for this CTA: nothing was taken yet
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * SL::kStage);
-    uint64_t* full_tma = bars;
-    uint64_t* full_bf = bars + kStages;
-    uint64_t* empty = bars + 2 * kStages;
-    uint64_t* acc_full = bars + 3 * kStages;
+    uint64_t* full_tma = bars;                  // [kStages] TMA bytes landed
+    uint64_t* full_bf = bars + kStages;         // [kStages] converted by all converter warps
+    uint64_t* empty = bars + 2 * kStages;       // [kStages] MMAs reading the stage are done
+    uint64_t* acc_full = bars + 3 * kStages;    // [2] accumulator complete
+    uint64_t* acc_empty = acc_full + 2;         // [2] accumulator read out by the epilogue
+    uint64_t* mma_done = acc_empty + 2;         // every issued MMA complete (teardown)
     auto sA = [&](int s) { return smem + s * SL::kStage; };
     auto sBbf = [&](int s) { return smem + s * SL::kStage + SL::kA; };
     auto sBq = [&](int s) { return smem + s * SL::kStage + SL::kA + SL::kBbf; };
@@ -126,10 +134,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&full_tma[s], 1);
-            tc::mbar_init(&full_bf[s], 32 * 4);
+            tc::mbar_init(&full_bf[s], kConvWarps);
             tc::mbar_init(&empty[s], 1);
         }
-        tc::mbar_init(acc_full, 1);
+        for (int b = 0; b < 2; ++b) {
+            tc::mbar_init(&acc_full[b], 1);
+            tc::mbar_init(&acc_empty[b], kEpiWarps);
+        }
+        tc::mbar_init(mma_done, 1);
         abort_flag = 0;
         tc::mbar_fence_init();
     }
@@ -138,7 +150,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc::prefetch_tmap(&tmB0);
         if (kDual) tc::prefetch_tmap(&tmB1);
     }
-    if (warp == 1) tc::tmem_alloc(&tmem_holder, BN);
+    if (warp == 1) tc::tmem_alloc(&tmem_holder, kTmemCols);
     tc::tc_fence_before();
     __syncthreads();
     tc::tc_fence_after();
@@ -150,84 +162,120 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int mma_issued = 0;
 
     if (warp == 0) {
+        // ---------------- TMA producer
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages, r = kb / kStages;
-                if (r > 0 && !tc::mbar_wait_bounded(&empty[s], (r - 1) & 1, &abort_flag, kMaxPolls)) {
-                    if (!abort_flag) fail(p.hdr, &abort_flag);
-                    break;
-                }
-                tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
-                tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
-                if (kDual) {
+            int g = 0;
+            TileCoord t;
+            for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x) {
+                tile_coord(hdr, p, L, t);
+                const int a_row0 = hdr->seg_start[t.e] + t.m_tile * kBM;
+                const int w_row0 = t.e * p.N + t.n_tile * (kDual ? BN / 2 : BN);
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStages, r = g / kStages;
+                    if (r > 0 && !tc::mbar_wait_bounded(&empty[s], (r - 1) & 1, &abort_flag, kMaxPolls)) {
+                        if (!abort_flag) fail(p.hdr, &abort_flag);
+                        ok = false;
+                        break;
+                    }
+                    tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
+                    tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
                     tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
-                    tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
-                } else {
-                    tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                    if (kDual) tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                    issued_round[s] = r;
                 }
-                issued_round[s] = r;
+                if (!ok) break;
             }
         }
     } else if (warp == 1) {
+        // ---------------- MMA issuer
         if (lane == 0) {
-            for (int kb = 0; kb < KB; ++kb) {
-                const int s = kb % kStages, r = kb / kStages;
-                if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls) ||
-                    !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, kMaxPolls)) {
+            int g = 0, it = 0;
+            for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x, ++it) {
+                const int b = it & 1, u = it >> 1;
+                if (u > 0 && !tc::mbar_wait_bounded(&acc_empty[b], (u - 1) & 1, &abort_flag, kMaxPolls)) {
                     if (!abort_flag) fail(p.hdr, &abort_flag);
                     break;
                 }
                 tc::tc_fence_after();
-                const uint64_t adesc = tc::sw128_kmajor_desc(tc::smem_u32(sA(s)));
-                const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sBbf(s)));
+                const uint32_t d_tmem = tmem + (uint32_t)(b * BN);
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int s = g % kStages, r = g / kStages;
+                    if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls) ||
+                        !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, kMaxPolls)) {
+                        if (!abort_flag) fail(p.hdr, &abort_flag);
+                        ok = false;
+                        break;
+                    }
+                    tc::tc_fence_after();
+                    const uint64_t adesc = tc::sw128_kmajor_desc(tc::smem_u32(sA(s)));
+                    const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sBbf(s)));
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per 16-element K step = +2 in the address field
-                    tc::mma_bf16_ss(tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
-                tc::mma_commit(&empty[s]);
-                ++mma_issued;
+                    for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per 16-element K step = +2 in the address field
+                        tc::mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+                    tc::mma_commit(&empty[s]);
+                    ++mma_issued;
+                }
+                if (!ok) break;
+                tc::mma_commit(&acc_full[b]);
             }
-            tc::mma_commit(acc_full);  // arrives once every MMA issued above has completed
+            tc::mma_commit(mma_done);  // arrives once every MMA issued above has completed
         }
         __syncwarp();
-    } else {
-        // ---- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte chunk c of row r
-        // stored at chunk c ^ (r & 7) of the row's 128 bytes)
+    } else if (warp < 2 + kConvWarps) {
+        // ---------------- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte
+        // chunk c of row r stored at chunk c ^ (r & 7) of the row's 128 bytes)
         const int t = threadIdx.x - 64;
-        for (int kb = 0; kb < KB; ++kb) {
-            const int s = kb % kStages, r = kb / kStages;
-            if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls)) {
-                if (!abort_flag) fail(p.hdr, &abort_flag);
-                break;
-            }
-            const uint8_t* q8 = sBq(s);
-            uint8_t* bf = sBbf(s);
+        int g = 0;
+        for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x) {
+            bool ok = true;
+            for (int kb = 0; kb < KB; ++kb, ++g) {
+                const int s = g % kStages, r = g / kStages;
+                if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls)) {
+                    if (!abort_flag) fail(p.hdr, &abort_flag);
+                    ok = false;
+                    break;
+                }
+                const uint8_t* q8 = sBq(s);
+                uint8_t* bf = sBbf(s);
 #pragma unroll
-            for (int i = 0; i < BN * 4 / 128; ++i) {
-                const int qi = t + 128 * i, row = qi >> 2, c = qi & 3;
-                const uint4 v = *reinterpret_cast<const uint4*>(q8 + row * kBK + c * 16);
-                uint32_t o[8];
-                convert16(v, o);
-                uint8_t* rp = bf + row * 128;
-                *reinterpret_cast<uint4*>(rp + (((2 * c) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<uint4*>(rp + (((2 * c + 1) ^ (row & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+                for (int i = 0; i < BN * 4 / (kConvWarps * 32); ++i) {
+                    const int qi = t + kConvWarps * 32 * i, row = qi >> 2, c = qi & 3;
+                    const uint4 v = *reinterpret_cast<const uint4*>(q8 + row * kBK + c * 16);
+                    uint32_t o[8];
+                    convert16(v, o);
+                    uint8_t* rp = bf + row * 128;
+                    *reinterpret_cast<uint4*>(rp + (((2 * c) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<uint4*>(rp + (((2 * c + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(o[4], o[5], o[6], o[7]);
+                }
+                tc::fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&full_bf[s]);
             }
-            tc::fence_proxy_async_smem();
-            tc::mbar_arrive(&full_bf[s]);
+            if (!ok) break;
         }
-        // ---- epilogue
-        bool ok = tc::mbar_wait_bounded(acc_full, 0, &abort_flag, kMaxPolls);
-        if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
-        ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
-        tc::tc_fence_after();
-        if (ok) {
-            const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 are this warp's
-            const int row = q * 32 + lane;
-            const int64_t gr = (int64_t)a_row0 + row;
-            const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16);
+    } else {
+        // ---------------- epilogue
+        const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
+        const int row = q * 32 + lane;
+        int it = 0;
+        TileCoord t;
+        for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x, ++it) {
+            const int b = it & 1, u = it >> 1;
+            bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, kMaxPolls);
+            if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
+            ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+            if (!ok) break;
+            tc::tc_fence_after();
+            tile_coord(hdr, p, L, t);
+            const int64_t gr = (int64_t)hdr->seg_start[t.e] + t.m_tile * kBM + row;
+            const uint32_t tbase = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
             if (kDual) {
-                const int j0 = n_tile * (BN / 2);
-                const float* s1 = p.sa + (int64_t)e * p.N + j0;
-                const float* s3 = p.sb + (int64_t)e * p.N + j0;
+                const int j0 = t.n_tile * (BN / 2);
+                const float* s1 = p.sa + (int64_t)t.e * p.N + j0;
+                const float* s3 = p.sb + (int64_t)t.e * p.N + j0;
                 uint16_t* hrow = p.h_out + gr * p.N + j0;
 #pragma unroll 1
                 for (int c = 0; c < BN / 2; c += 32) {
@@ -251,10 +299,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                 }
             } else {
-                const int i0 = n_tile * BN;
+                const int i0 = t.n_tile * BN;
                 const int32_t a = p.perm[gr];
                 const float wt = a >= 0 ? p.wts[a] : 0.0f;
-                const float* s2 = p.sa + (int64_t)e * p.N + i0;
+                const float* s2 = p.sa + (int64_t)t.e * p.N + i0;
                 float* orow = p.slot_out + (int64_t)(a >= 0 ? a : 0) * p.N + i0;
 #pragma unroll 1
                 for (int c = 0; c < BN; c += 32) {
@@ -275,6 +323,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
         }
     }
 
@@ -285,19 +336,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (warp == 0 && lane == 0) {
             for (int s = 0; s < kStages; ++s) {
                 if (issued_round[s] < 0) continue;
-                // a copy of round r completes phase r of full_tma[s]; waiting ignores the abort flag
+                // a copy of round r completes phase r of full_tma[s]; this wait ignores the abort flag
                 for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(&full_tma[s], issued_round[s] & 1); ++i)
                     __nanosleep(64);
             }
         }
         if (warp == 1 && lane == 0 && mma_issued > 0) {
-            for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(acc_full, 0); ++i) __nanosleep(64);
+            for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(mma_done, 0); ++i) __nanosleep(64);
         }
         __syncthreads();
     }
     if (warp == 1) {
         tc::tc_fence_after();
-        tc::tmem_dealloc(tmem, BN);
+        tc::tmem_dealloc(tmem, kTmemCols);
     }
 }
 
@@ -349,7 +400,15 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SL::kSmem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = m_tiles_cap * p.n_tiles;
+    // persistent: one CTA per SM (fewer when there are fewer tile slots)
+    static int sms_cache[64] = {0};
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
+        if (!sms_cache[dev]) cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (sms_cache[dev] > 0) sms = sms_cache[dev];
+    }
+    int64_t grid = m_tiles_cap * p.n_tiles;
+    if (grid > sms) grid = sms;
     gemm_tc_kernel<kDual, BN><<<(unsigned)grid, kGemmThreads, SL::kSmem, st>>>(ta, tb0, tb1, p);
     return cudaGetLastError();
 }
