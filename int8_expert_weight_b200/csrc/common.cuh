@@ -58,14 +58,31 @@ __device__ __forceinline__ uint32_t bf16x2_v_minus_c(uint32_t v, uint32_t c) {
     asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(c), "r"(0xBF80BF80u), "r"(v));
     return r;
 }
+// The three bit masks of the conversion, held in registers: as immediates the compiler splits each
+// (w & mask) | exponent into two logic instructions; with all operands in registers it is one lop3.
+struct S8Consts {
+    uint32_t low7, sign, expo;
+};
+__device__ __forceinline__ S8Consts s8_consts() {
+    S8Consts k;
+    asm volatile("mov.b32 %0, 0x007F007F;" : "=r"(k.low7));
+    asm volatile("mov.b32 %0, 0x00800080;" : "=r"(k.sign));
+    asm volatile("mov.b32 %0, 0x43004300;" : "=r"(k.expo));
+    return k;
+}
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {  // (a & b) | c
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
 // Bytes 0 and 2 of a 32-bit word as a bf16x2 (byte 0 in the low half).
-__device__ __forceinline__ uint32_t s8x2_even_to_bf16x2(uint32_t w) {
-    const uint32_t v = (w & 0x007F007Fu) | 0x43004300u;
-    const uint32_t c = (w & 0x00800080u) | 0x43004300u;
-    return bf16x2_v_minus_c(v, c);
+__device__ __forceinline__ uint32_t s8x2_even_to_bf16x2(uint32_t w, const S8Consts& k) {
+    return bf16x2_v_minus_c(and_or(w, k.low7, k.expo), and_or(w, k.sign, k.expo));
 }
 // Bytes 1 and 3 of the word.
-__device__ __forceinline__ uint32_t s8x2_odd_to_bf16x2(uint32_t w) { return s8x2_even_to_bf16x2(w >> 8); }
+__device__ __forceinline__ uint32_t s8x2_odd_to_bf16x2(uint32_t w, const S8Consts& k) {
+    return s8x2_even_to_bf16x2(w >> 8, k);
+}
 
 // bf16 pairs (e0, e2) and (e1, e3) from two bf16x2 words holding (e0, e1) and (e2, e3).
 __device__ __forceinline__ uint32_t pair_lo(uint32_t a, uint32_t b) { return __byte_perm(a, b, 0x5410); }

@@ -228,11 +228,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // chunk c of row r stored at chunk c ^ (r & 7) of the row's 128 bytes)
         const int t = threadIdx.x - 64;
         int g = 0;
-        for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x) {
+        for (int L = blockIdx.x; L < total; L += gridDim.x) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % kStages, r = g / kStages;
-                if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls)) {
+                const bool landed = tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls);
+                if (!__all_sync(0xffffffffu, landed)) {  // warp-uniform: __syncwarp below needs all lanes
                     if (!abort_flag) fail(p.hdr, &abort_flag);
                     ok = false;
                     break;
@@ -262,7 +264,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int row = q * 32 + lane;
         int it = 0;
         TileCoord t;
-        for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x, ++it) {
+        for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
+            if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
             const int b = it & 1, u = it >> 1;
             bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, kMaxPolls);
             if (!ok && !abort_flag) fail(p.hdr, &abort_flag);

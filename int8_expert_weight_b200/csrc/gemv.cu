@@ -48,13 +48,13 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int j) {
 
 template <int NT, bool kDual>
 __device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[NT][4], const WeightRegs<kDual>& w,
-                                         const uint4 (&xa)[NT][2]) {
+                                         const uint4 (&xa)[NT][2], const S8Consts& k) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         // A fragment: k positions (2c, 2c+1) <- bytes 4j, 4j+2; (2c+8, 2c+9) <- bytes 4j+1, 4j+3.
         const uint32_t wa0 = word(w.a0, j), wa1 = word(w.a1, j);
-        const uint32_t a0 = s8x2_even_to_bf16x2(wa0), a1 = s8x2_even_to_bf16x2(wa1);
-        const uint32_t a2 = s8x2_odd_to_bf16x2(wa0), a3 = s8x2_odd_to_bf16x2(wa1);
+        const uint32_t a0 = s8x2_even_to_bf16x2(wa0, k), a1 = s8x2_even_to_bf16x2(wa1, k);
+        const uint32_t a2 = s8x2_odd_to_bf16x2(wa0, k), a3 = s8x2_odd_to_bf16x2(wa1, k);
         uint32_t b0[NT], b1[NT];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -68,8 +68,8 @@ __device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[N
         }
         if (kDual) {
             const uint32_t wb0 = word(w.b0, j), wb1 = word(w.b1, j);
-            const uint32_t c0 = s8x2_even_to_bf16x2(wb0), c1 = s8x2_even_to_bf16x2(wb1);
-            const uint32_t c2 = s8x2_odd_to_bf16x2(wb0), c3 = s8x2_odd_to_bf16x2(wb1);
+            const uint32_t c0 = s8x2_even_to_bf16x2(wb0, k), c1 = s8x2_even_to_bf16x2(wb1, k);
+            const uint32_t c2 = s8x2_odd_to_bf16x2(wb0, k), c3 = s8x2_odd_to_bf16x2(wb1, k);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc_b[nt], c0, c1, c2, c3, b0[nt], b1[nt]);
         }
@@ -104,6 +104,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
         for (int i = 0; i < 4; ++i) acc_a[nt][i] = acc_b[nt][i] = 0.0f;
 
     const int steps = (int)(K / 64);
+    const S8Consts k = s8_consts();
     for (int s0 = warp; s0 < steps; s0 += kGemvWarps * U) {
         WeightRegs<kDual> w[U];
         uint4 xa[U][NT][2];
@@ -125,7 +126,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (s0 + u * kGemvWarps < steps) mma_step<NT, kDual>(acc_a, acc_b, w[u], xa[u]);
+            if (s0 + u * kGemvWarps < steps) mma_step<NT, kDual>(acc_a, acc_b, w[u], xa[u], k);
         pa0 += U * kStride;
         pa1 += U * kStride;
         if (kDual) {
@@ -156,7 +157,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
 }
 
 template <int NT, bool kDual>
-__global__ void __launch_bounds__(kGemvWarps * 32, (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
+__global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1 && kDual) ? 3 : (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
     const WsHeader* hdr = p.hdr;
     if ((int)blockIdx.y >= hdr->n_touched) return;
