@@ -57,19 +57,22 @@ struct StageLayout {
     static constexpr int kSmem = kStages * kStage + 1024 + 256;
 };
 
-// bf16x2 of two bytes of w, exactly, in k order: (0x4300 | low 7 bits) - (0x4300 | sign bit).
-__device__ __forceinline__ uint32_t s8pair_to_bf16x2(uint32_t lo7, uint32_t hi1, uint32_t sel) {
-    return bf16x2_v_minus_c(__byte_perm(lo7, 0x43434343u, sel), __byte_perm(hi1, 0x43434343u, sel));
-}
-
-__device__ __forceinline__ void convert16(const uint4 v, uint32_t (&o)[8]) {
+// 16 int8 weights -> 8 bf16x2 words, exactly.  Word i of the input (bytes b0..b3) yields the pairs
+// (b0, b2) and (b1, b3), so within every group of 4 the stored k order is 0, 2, 1, 3; the
+// activation operands of this path are stored with the same order (elements 1 and 2 of each group
+// of 4 swapped), and a k-permutation applied to both operands leaves every dot product unchanged.
+__device__ __forceinline__ void convert16(const uint4 v, uint32_t (&o)[8], const S8Consts& k) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t lo7 = w[i] & 0x7F7F7F7Fu, hi1 = w[i] & 0x80808080u;
-        o[2 * i] = s8pair_to_bf16x2(lo7, hi1, 0x4140);      // bytes 0, 1
-        o[2 * i + 1] = s8pair_to_bf16x2(lo7, hi1, 0x4342);  // bytes 2, 3
+        o[2 * i] = s8x2_even_to_bf16x2(w[i], k);
+        o[2 * i + 1] = s8x2_odd_to_bf16x2(w[i], k);
     }
+}
+
+// Swap elements 1 and 2 of a group of 4 bf16 held as two bf16x2 words (lo = e0 e1, hi = e2 e3).
+__device__ __forceinline__ uint2 swap_mid4(uint32_t lo, uint32_t hi) {
+    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
 }
 
 __device__ __forceinline__ void fail(WsHeader* hdr, volatile int* abort) {
@@ -227,6 +230,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---------------- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte
         // chunk c of row r stored at chunk c ^ (r & 7) of the row's 128 bytes)
         const int t = threadIdx.x - 64;
+        const S8Consts k8 = s8_consts();
         int g = 0;
         for (int L = blockIdx.x; L < total; L += gridDim.x) {
             if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const int qi = t + kConvWarps * 32 * i, row = qi >> 2, c = qi & 3;
                     const uint4 v = *reinterpret_cast<const uint4*>(q8 + row * kBK + c * 16);
                     uint32_t o[8];
-                    convert16(v, o);
+                    convert16(v, o, k8);
                     uint8_t* rp = bf + row * 128;
                     *reinterpret_cast<uint4*>(rp + (((2 * c) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
                     *reinterpret_cast<uint4*>(rp + (((2 * c + 1) ^ (row & 7)) << 4)) =
@@ -296,10 +300,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         packed[i / 2] = (uint32_t)f32_to_bf16_bits(silu(g0) * u0) |
                                         ((uint32_t)f32_to_bf16_bits(silu(g1) * u1) << 16);
                     }
+                    // h feeds the down-projection GEMM as its activation operand: store every group of
+                    // 4 columns in the 0, 2, 1, 3 order that GEMM's weight conversion produces
                     uint4* dst = reinterpret_cast<uint4*>(hrow + c);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                    for (int v = 0; v < 4; ++v) {
+                        const uint2 a = swap_mid4(packed[4 * v], packed[4 * v + 1]);
+                        const uint2 b = swap_mid4(packed[4 * v + 2], packed[4 * v + 3]);
+                        dst[v] = make_uint4(a.x, a.y, b.x, b.y);
+                    }
                 }
             } else {
                 const int i0 = t.n_tile * BN;

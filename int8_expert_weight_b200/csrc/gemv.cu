@@ -157,7 +157,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
 }
 
 template <int NT, bool kDual>
-__global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1 && kDual) ? 3 : (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
+__global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
     const WsHeader* hdr = p.hdr;
     if ((int)blockIdx.y >= hdr->n_touched) return;
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1 && kDual) ? 3 : (NT 
                 rows[nt] = p.act + (row0 + nn) * p.K;
             }
         }
-        gemv_pass<NT, kDual, (kDual ? 2 : 4)>(p, e, j0, rows, red);
+        gemv_pass<NT, kDual, 2>(p, e, j0, rows, red);
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
         for (int o = threadIdx.x; o < NT * 128; o += blockDim.x) {

@@ -94,8 +94,9 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
         for (int r = seg[e] + hist[e] + tid; r < seg[e + 1]; r += kPermThreads) perm[r] = -1;
 }
 
-// x_perm[r] = x[perm[r] / K] for real rows, zeros for padding rows; rows past the last segment
-// are left alone.  16-byte vector copies, one warp per row.
+// x_perm[r] = x[perm[r] / K] for real rows (elements 1 and 2 of every group of 4 swapped, the k
+// order of the tensor-core path), zeros for padding rows; rows past the last segment are left
+// alone.  16-byte vector copies, one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ perm,
                                                           const WsHeader* __restrict__ hdr, int64_t d,
@@ -109,8 +110,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         if (a < 0) {
             for (int64_t c = lane; c < chunks; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
         } else {
+            // elements 1 and 2 of every group of 4 swapped: the k order of the GEMM path's weights
             const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(a / kTopK) * d);
-            for (int64_t c = lane; c < chunks; c += 32) dst[c] = ld_nc_v4(src + c);
+            for (int64_t c = lane; c < chunks; c += 32) {
+                const uint4 v = ld_nc_v4(src + c);
+                dst[c] = make_uint4(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632),
+                                    __byte_perm(v.z, v.w, 0x5410), __byte_perm(v.z, v.w, 0x7632));
+            }
         }
     }
 }
