@@ -257,6 +257,28 @@ def l2_note(wl):
     return "inputs fit in L2 (%.1f MB): not a roofline workload" % (wbytes / 1e6)
 
 
+# ------------------------------------------------------------------ multi-rank helpers
+def rank_seed(wl, rank):
+    """Each rank draws its own batch of tokens (weak scaling); weights use the workload seed."""
+    return wl.seed + rank
+
+
+def max_over_ranks(value, device):
+    """The largest value over all ranks (one all-reduce); the value itself with one process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tokens_per_s(world, T, steps, max_ms):
+    """Whole-job throughput: every rank processed T tokens per step; time = slowest rank."""
+    return world * T * steps / (max_ms / 1e3)
+
+
 # ------------------------------------------------------------------ the CUDA arm
 def run_ours(args):
     import torch
@@ -276,7 +298,7 @@ def run_ours(args):
     peaks = load_peaks()
 
     # ---- inputs: this rank's batch (own seed), replicated weights quantized by the library (load time)
-    seed_x = wl.seed + rank
+    seed_x = rank_seed(wl, rank)
     x_bits = synth.gen_x(synth_replace(wl, seed=seed_x))
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa
     x = to_dev(x_bits)
@@ -336,12 +358,8 @@ def run_ours(args):
         barrier()
         kernels = jm.jamba_moe_timing_collect()
         jm.jamba_moe_timing_start(0)
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * T * args.steps / (ms / 1e3)
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    value = aggregate_tokens_per_s(world, T, args.steps, ms)
 
     # ---- end to end through the public call with host buffers: pinned x in, pinned y out
     x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
@@ -364,12 +382,8 @@ def run_ours(args):
         step_e2e()
     ev1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
+    e2e_value = aggregate_tokens_per_s(world, T, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     dom = max(kernels, key=lambda k: kernels[k][0])
