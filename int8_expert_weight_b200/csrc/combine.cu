@@ -8,6 +8,8 @@ namespace jmoe {
 
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ slots, int64_t T, int64_t d,
                                                       uint16_t* __restrict__ y) {
+    pdl_wait();
+    pdl_trigger();
     const int64_t quads = T * d / 4;  // d % 4 == 0
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < quads; q += stride) {
@@ -24,8 +26,7 @@ cudaError_t launch_combine(const float* slots, int64_t T, int64_t d, uint16_t* y
     int64_t blocks = (T * d / 4 + 255) / 256;
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     if (blocks < 1) blocks = 1;
-    combine_kernel<<<(unsigned)blocks, 256, 0, st>>>(slots, T, d, y);
-    return cudaGetLastError();
+    return launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(256), 0, st, slots, T, d, y);
 }
 
 }  // namespace jmoe

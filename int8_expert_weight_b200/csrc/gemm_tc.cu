@@ -117,6 +117,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
 
+    pdl_wait();
     const WsHeader* hdr = p.hdr;
     const int total = hdr->tile_start[kExperts] * p.n_tiles;
     if ((int)blockIdx.x >= total) return;  // no tile for this CTA: nothing was taken yet
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
 
     // ---- teardown: after an abort, let in-flight copies and MMAs finish (bounded) before TMEM goes
+    pdl_trigger();
     tc::tc_fence_before();
     __syncthreads();
     if (abort_flag) {
@@ -421,8 +423,8 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
     }
     int64_t grid = m_tiles_cap * p.n_tiles;
     if (grid > sms) grid = sms;
-    gemm_tc_kernel<kDual, BN><<<(unsigned)grid, kGemmThreads, SL::kSmem, st>>>(ta, tb0, tb1, p);
-    return cudaGetLastError();
+    return launch_pdl(gemm_tc_kernel<kDual, BN>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta, tb0,
+                      tb1, p);
 }
 
 }  // namespace

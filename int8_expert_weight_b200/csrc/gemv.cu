@@ -159,6 +159,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
 template <int NT, bool kDual>
 __global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
+    pdl_wait();
     const WsHeader* hdr = p.hdr;
     if ((int)blockIdx.y >= hdr->n_touched) return;
     const int e = hdr->touched[blockIdx.y];
@@ -181,6 +182,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4)
             }
         }
         gemv_pass<NT, kDual, 2>(p, e, j0, rows, red);
+        pdl_trigger();  // main loop done: the next kernel may start launching
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
         for (int o = threadIdx.x; o < NT * 128; o += blockDim.x) {
@@ -210,13 +212,9 @@ static int gemv_nt(int64_t T) {
 template <bool kDual>
 static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st) {
     dim3 grid((unsigned)(p.N / kGemvRows), kExperts);
-    if (nt == 1)
-        gemv_kernel<1, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
-    else if (nt == 2)
-        gemv_kernel<2, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
-    else
-        gemv_kernel<4, kDual><<<grid, kGemvWarps * 32, 0, st>>>(p);
-    return cudaGetLastError();
+    if (nt == 1) return launch_pdl(gemv_kernel<1, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
+    if (nt == 2) return launch_pdl(gemv_kernel<2, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
+    return launch_pdl(gemv_kernel<4, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
 }
 
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,

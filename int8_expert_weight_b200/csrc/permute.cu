@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
     __shared__ int wcount[kPermThreads / 32][kExperts];
     __shared__ int wpre[kPermThreads / 32][kExperts];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    pdl_trigger();
     if (tid < kExperts) hist[tid] = 0;
     if (tid == 0) hdr->status = 0;  // first kernel of a forward call to touch the header
     __syncthreads();
@@ -102,6 +104,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const WsHeader* __restrict__ hdr, int64_t d,
                                                           int64_t cap_rows, uint16_t* __restrict__ x_perm) {
     const int lane = threadIdx.x & 31;
+    pdl_wait();
+    pdl_trigger();
     const int64_t nrows = min((int64_t)hdr->seg_start[kExperts], cap_rows);
     const int64_t chunks = d / 8;
     for (int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5); r < nrows; r += (int64_t)gridDim.x * 8) {
@@ -123,8 +127,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 
 cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
                            cudaStream_t st) {
-    permute_kernel<<<1, kPermThreads, 0, st>>>(ids, T * kTopK, hdr, perm, inv);
-    return cudaGetLastError();
+    return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), 0, st, ids, T * kTopK, hdr, perm, inv);
 }
 
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
@@ -132,8 +135,8 @@ cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader
     int64_t blocks = (cap_rows + 7) / 8;
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     if (blocks < 1) blocks = 1;
-    gather_rows_kernel<<<(unsigned)blocks, 256, 0, st>>>(x, perm, hdr, d, cap_rows, x_perm);
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, perm, hdr, d, cap_rows,
+                      x_perm);
 }
 
 }  // namespace jmoe

@@ -58,6 +58,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(const uint16_t* 
                                                                 float* __restrict__ w_user) {
     __shared__ float red[kRouterThreads][kRouterTokens * kExperts + 1];
     __shared__ float logits[kRouterTokens][kExperts];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x;
     const int64_t t0 = (int64_t)blockIdx.x * kRouterTokens;
 
@@ -118,6 +120,8 @@ __global__ void __launch_bounds__(kRouterSmallThreads) router_token_kernel(
     float* __restrict__ w_user) {
     __shared__ float part[kRouterSmallThreads / 32][kExperts];
     __shared__ float logits[kExperts];
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t t = blockIdx.x;
     float acc[kExperts];
@@ -165,12 +169,12 @@ __global__ void __launch_bounds__(kRouterSmallThreads) router_token_kernel(
 cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias, int64_t T, int64_t d,
                           int32_t* ids_ws, float* w_ws, int32_t* ids_user, float* w_user, cudaStream_t st) {
     if (T <= 512) {
-        router_token_kernel<<<(unsigned)T, kRouterSmallThreads, 0, st>>>(x, Wr, bias, d, ids_ws, w_ws, ids_user,
-                                                                          w_user);
+        return launch_pdl(router_token_kernel, dim3((unsigned)T), dim3(kRouterSmallThreads), 0, st, x, Wr, bias, d,
+                          ids_ws, w_ws, ids_user, w_user);
     } else {
         const int64_t blocks = (T + kRouterTokens - 1) / kRouterTokens;
-        router_kernel<<<(unsigned)blocks, kRouterThreads, 0, st>>>(x, Wr, bias, T, d, ids_ws, w_ws, ids_user,
-                                                                    w_user);
+        return launch_pdl(router_kernel, dim3((unsigned)blocks), dim3(kRouterThreads), 0, st, x, Wr, bias, T, d,
+                          ids_ws, w_ws, ids_user, w_user);
     }
     return cudaGetLastError();
 }
