@@ -133,6 +133,17 @@ int jamba_moe_read_device_status(const void* workspace, void* stream);
 const char* jamba_moe_status_string(int status);
 
 /*
+ * jamba_moe_debug_skip_copy — test hook for failure detection, off by default.  While `on` is
+ * non-zero, the next forward calls on the tensor-core (prefill) path make CTA 0 of the W1/W3 GEMM
+ * skip the copies of its second K step, with every pipeline wait bounded by a short poll limit:
+ * the wait for those copies runs out, the kernel records JMOE_DEV_TIMEOUT in the workspace status
+ * word, waits (bounded) for its other in-flight copies and MMAs, releases its tensor memory and
+ * returns; the output of that call is not valid.  Nothing faults, traps or hangs, and the CUDA
+ * context stays usable.  Host only; not thread-safe.
+ */
+int jamba_moe_debug_skip_copy(int on);
+
+/*
  * jamba_moe_forward_noalloc — jamba_moe_forward on the decode (weight-streaming) path for callers
  * that cannot allocate device memory: code running inside a memory pool it does not own, a
  * serving process that must not call cudaMalloc after start-up (it synchronises the device and

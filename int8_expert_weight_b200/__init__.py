@@ -65,6 +65,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_noalloc_scratch_capacity.argtypes = []
     lib.jamba_moe_noalloc_scratch_needed.restype = sz
     lib.jamba_moe_noalloc_scratch_needed.argtypes = [i64, i64, i64]
+    lib.jamba_moe_debug_skip_copy.restype = c_int
+    lib.jamba_moe_debug_skip_copy.argtypes = [c_int]
     lib.jamba_moe_kernel_name.restype = ctypes.c_char_p
     lib.jamba_moe_kernel_name.argtypes = [c_int]
     _lib = lib
@@ -206,6 +208,11 @@ def jamba_moe_read_device_status(workspace: torch.Tensor, stream: Optional[torch
     """Synchronise the stream and return the device status word of the last forward on workspace."""
     _check(workspace, "workspace", torch.uint8)
     return int(load_library().jamba_moe_read_device_status(workspace.data_ptr(), _stream_ptr(stream)))
+
+
+def jamba_moe_debug_skip_copy(on: bool) -> None:
+    """Test hook (see include/jmoe.h): make one tensor-core pipeline wait run out on purpose."""
+    load_library().jamba_moe_debug_skip_copy(1 if on else 0)
 
 
 def jamba_moe_timing_start(max_launches: int) -> None:

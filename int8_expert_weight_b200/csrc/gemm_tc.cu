@@ -32,7 +32,8 @@ constexpr int kStages = 3;
 constexpr int kConvWarps = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kGemmThreads = (2 + kConvWarps + kEpiWarps) * 32;
-constexpr uint32_t kMaxPolls = 1u << 22;
+constexpr uint32_t kMaxPolls = 1u << 22;       // ~0.3 s of polling: far above any healthy wait
+constexpr uint32_t kTestMaxPolls = 1u << 14;   // short bound used together with the test hook
 
 struct GemmArgs {
     WsHeader* hdr;
@@ -46,6 +47,8 @@ struct GemmArgs {
     int N;                // weight rows per expert and matrix: ffn (gemm13) or d (gemm2)
     int n_tiles;          // N tiles per M tile
     int band;             // M tiles per raster band
+    uint32_t max_polls;   // bound of every mbarrier wait
+    int skip_copy;        // test hook: CTA 0 skips the copies of its second K step (a wait then runs out)
 };
 
 template <int BN>
@@ -177,11 +180,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages, r = g / kStages;
-                    if (r > 0 && !tc::mbar_wait_bounded(&empty[s], (r - 1) & 1, &abort_flag, kMaxPolls)) {
+                    if (r > 0 && !tc::mbar_wait_bounded(&empty[s], (r - 1) & 1, &abort_flag, p.max_polls)) {
                         if (!abort_flag) fail(p.hdr, &abort_flag);
                         ok = false;
                         break;
                     }
+                    if (p.skip_copy && blockIdx.x == 0 && L == (int)blockIdx.x && kb == 1) continue;
                     tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
                     tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
                     tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
@@ -197,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             int g = 0, it = 0;
             for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x, ++it) {
                 const int b = it & 1, u = it >> 1;
-                if (u > 0 && !tc::mbar_wait_bounded(&acc_empty[b], (u - 1) & 1, &abort_flag, kMaxPolls)) {
+                if (u > 0 && !tc::mbar_wait_bounded(&acc_empty[b], (u - 1) & 1, &abort_flag, p.max_polls)) {
                     if (!abort_flag) fail(p.hdr, &abort_flag);
                     break;
                 }
@@ -206,8 +210,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages, r = g / kStages;
-                    if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls) ||
-                        !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, kMaxPolls)) {
+                    if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls) ||
+                        !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, p.max_polls)) {
                         if (!abort_flag) fail(p.hdr, &abort_flag);
                         ok = false;
                         break;
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++g) {
                 const int s = g % kStages, r = g / kStages;
-                const bool landed = tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, kMaxPolls);
+                const bool landed = tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls);
                 if (!__all_sync(0xffffffffu, landed)) {  // warp-uniform: __syncwarp below needs all lanes
                     if (!abort_flag) fail(p.hdr, &abort_flag);
                     ok = false;
@@ -272,7 +276,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
             if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
             const int b = it & 1, u = it >> 1;
-            bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, kMaxPolls);
+            bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, p.max_polls);
             if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
             ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
             if (!ok) break;
@@ -351,12 +355,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int s = 0; s < kStages; ++s) {
                 if (issued_round[s] < 0) continue;
                 // a copy of round r completes phase r of full_tma[s]; this wait ignores the abort flag
-                for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(&full_tma[s], issued_round[s] & 1); ++i)
+                for (uint32_t i = 0; i < p.max_polls && !tc::mbar_try_wait(&full_tma[s], issued_round[s] & 1); ++i)
                     __nanosleep(64);
             }
         }
         if (warp == 1 && lane == 0 && mma_issued > 0) {
-            for (uint32_t i = 0; i < kMaxPolls && !tc::mbar_try_wait(mma_done, 0); ++i) __nanosleep(64);
+            for (uint32_t i = 0; i < p.max_polls && !tc::mbar_try_wait(mma_done, 0); ++i) __nanosleep(64);
         }
         __syncthreads();
     }
@@ -400,6 +404,8 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int g_skip_copy = 0;  // set by jamba_moe_debug_skip_copy (tests only)
+
 int band_for(int K) {
     // keep a band's activation tiles (band * 128 rows * K * 2 bytes) near 24 MB of L2
     const int64_t per_tile = (int64_t)kBM * K * 2;
@@ -441,7 +447,10 @@ cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_
         !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, kBK,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    GemmArgs p{hdr, perm, S1, S3, nullptr, h, nullptr, (int)d, (int)F, (int)(F / 128), band_for((int)d)};
+    GemmArgs p{hdr,          perm,          S1,          S3,
+               nullptr,      h,             nullptr,     (int)d,
+               (int)F,       (int)(F / 128), band_for((int)d), g_skip_copy ? kTestMaxPolls : kMaxPolls,
+               g_skip_copy};
     return launch_gemm_t<true, 256>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
@@ -454,9 +463,20 @@ cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, 
         !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * d, F, BN, kBK,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    GemmArgs p{hdr, perm, S2, nullptr, wts, nullptr, out_slot, (int)F, (int)d, (int)(d / BN), band_for((int)F)};
+    GemmArgs p{hdr,         perm,         S2,          nullptr,
+               wts,         nullptr,      out_slot,    (int)F,
+               (int)d,      (int)(d / BN), band_for((int)F), g_skip_copy ? kTestMaxPolls : kMaxPolls,
+               0};
     if (BN == 256) return launch_gemm_t<false, 256>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
 
 }  // namespace jmoe
+
+// Test hook: while `on` is non-zero, the W1/W3 tensor-core GEMM's CTA 0 skips the copies of its
+// second K step, so the pipeline wait for them runs out (after a short bound) and the kernel must
+// report JMOE_DEV_TIMEOUT, release its resources and return.  Nothing faults or hangs.
+extern "C" int jamba_moe_debug_skip_copy(int on) {
+    jmoe::g_skip_copy = on ? 1 : 0;
+    return JMOE_OK;
+}
