@@ -42,6 +42,9 @@ class Oracle:
         lib.oracle_moe_forward.restype = c_int
         lib.oracle_moe_forward.argtypes = [vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp,
                                            vp, i64, vp, vp, vp, vp, c_int]
+        lib.oracle_moe_forward_bf16w.restype = c_int
+        lib.oracle_moe_forward_bf16w.argtypes = [vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, i64, vp,
+                                                 vp, vp, vp, c_int]
         lib.oracle_default_threads.restype = c_int
         lib.oracle_default_threads.argtypes = []
         self.lib = lib
@@ -114,6 +117,33 @@ class Oracle:
             out["h"] = h
         return out
 
+    def moe_forward_bf16w(self, x_bits, router_w, bias, w1, w3, w2, tokens=None, top_k: int = 2,
+                          threads: int = 0, want_hidden: bool = False):
+        """The layer in fp64 with unquantized bf16 weights (uint16 bit patterns): w1, w3 [E][F][d],
+        w2 [E][d][F]; other arguments and the result as in moe_forward."""
+        x = _c(x_bits, np.uint16)
+        wr = _c(router_w, np.float32)
+        b = _c(bias, np.float32)
+        w1, w3, w2 = (_c(a, np.uint16) for a in (w1, w3, w2))
+        T, d = x.shape
+        E, F = w1.shape[0], w1.shape[1]
+        assert w1.shape == (E, F, d) and w3.shape == (E, F, d) and w2.shape == (E, d, F) and wr.shape == (E, d)
+        tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+        n = T if tok is None else tok.size
+        y = np.empty((n, d), dtype=np.float64)
+        ids = np.empty((n, top_k), dtype=np.int32)
+        wts = np.empty((n, top_k), dtype=np.float64)
+        h = np.empty((n, top_k, F), dtype=np.float64) if want_hidden else None
+        rc = self.lib.oracle_moe_forward_bf16w(x.ctypes.data, T, d, F, E, top_k, wr.ctypes.data, _ptr(b),
+                                               w1.ctypes.data, w3.ctypes.data, w2.ctypes.data, _ptr(tok), n,
+                                               y.ctypes.data, ids.ctypes.data, wts.ctypes.data, _ptr(h), threads)
+        if rc != 0:
+            raise ValueError("oracle_moe_forward_bf16w rejected its arguments")
+        out = {"y": y, "ids": ids, "w": wts}
+        if want_hidden:
+            out["h"] = h
+        return out
+
 
 _default: Optional[Oracle] = None
 
@@ -139,3 +169,7 @@ def route(x_bits, router_w, bias=None, top_k: int = 2, threads: int = 0, want_lo
 
 def moe_forward(*args, **kwargs):
     return get().moe_forward(*args, **kwargs)
+
+
+def moe_forward_bf16w(*args, **kwargs):
+    return get().moe_forward_bf16w(*args, **kwargs)

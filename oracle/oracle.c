@@ -20,6 +20,8 @@
  *     the K largest logits in descending order (equal logits: lower expert
  *     index first), weights = the softmax probabilities of the chosen experts,
  *     not renormalised.
+ *   - oracle_moe_forward_bf16w: the same layer with unquantized bf16 weights (the comparator the
+ *     Jamba-1.5 paper measures ExpertsInt8 against in §3.1), weights taken as their exact values.
  *   - oracle_moe_forward: y_t = sum_k w_tk * E_{e_tk}(x_t) with SwiGLU experts
  *     E_e(x) = W2_e (SiLU(W1_e x) * (W3_e x)) (GLU variants, Shazeer 2020,
  *     cited by the Jamba paper), where each weight is the dequantized value
@@ -299,6 +301,93 @@ int oracle_moe_forward(const uint16_t* x, int64_t T, int64_t d, int64_t F, int E
     }
     fwd_ctx c = {x, d, F, E, K, wr, bias, q1, q3, q2, s1, s3, s2, tokens, y, ids, wts, h_out};
     parallel_for(n_tokens, threads, forward_range, &c);
+    return 0;
+}
+
+/* ------------------------------------------------------- bf16-weight layer */
+
+typedef struct {
+    const uint16_t* x;
+    int64_t d, F;
+    int E, K;
+    const float* wr;
+    const float* bias;
+    const uint16_t *w1, *w3, *w2;
+    const int64_t* tokens;
+    double* y;
+    int32_t* ids;
+    double* wts;
+    double* h_out;
+} fwdb_ctx;
+
+/* One SwiGLU expert on one token with bf16 weights (exact as doubles). */
+static void expert_ffn_bf16w(const fwdb_ctx* c, int e, const double* xd, double* h, double* o) {
+    const int64_t d = c->d, F = c->F;
+    const uint16_t* w1 = c->w1 + (int64_t)e * F * d;
+    const uint16_t* w3 = c->w3 + (int64_t)e * F * d;
+    const uint16_t* w2 = c->w2 + (int64_t)e * d * F;
+    for (int64_t j = 0; j < F; ++j) {
+        double a1 = 0.0, a3 = 0.0;
+        const uint16_t* r1 = w1 + j * d;
+        const uint16_t* r3 = w3 + j * d;
+        for (int64_t i = 0; i < d; ++i) {
+            a1 += (double)bf16_value(r1[i]) * xd[i];
+            a3 += (double)bf16_value(r3[i]) * xd[i];
+        }
+        h[j] = a1 / (1.0 + exp(-a1)) * a3;
+    }
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        const uint16_t* r2 = w2 + i * F;
+        for (int64_t j = 0; j < F; ++j) acc += (double)bf16_value(r2[j]) * h[j];
+        o[i] = acc;
+    }
+}
+
+static void forward_bf16w_range(void* p, int64_t b, int64_t e) {
+    fwdb_ctx* c = (fwdb_ctx*)p;
+    const int64_t d = c->d, F = c->F;
+    double* xd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    int32_t ids[64];
+    double wts[64];
+    for (int64_t n = b; n < e; ++n) {
+        const int64_t t = c->tokens ? c->tokens[n] : n;
+        const uint16_t* xt = c->x + t * d;
+        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);
+        route_token(xt, d, c->wr, c->bias, c->E, c->K, ids, wts, NULL);
+        double* yt = c->y + n * d;
+        for (int64_t i = 0; i < d; ++i) yt[i] = 0.0;
+        for (int k = 0; k < c->K; ++k) {
+            expert_ffn_bf16w(c, ids[k], xd, h, o);
+            for (int64_t i = 0; i < d; ++i) yt[i] += wts[k] * o[i];
+            if (c->h_out) memcpy(c->h_out + (n * c->K + k) * F, h, sizeof(double) * (size_t)F);
+            if (c->ids) c->ids[n * c->K + k] = ids[k];
+            if (c->wts) c->wts[n * c->K + k] = wts[k];
+        }
+    }
+    free(xd);
+    free(h);
+    free(o);
+}
+
+/* The layer with bf16 weights w1, w3 [E][F][d] and w2 [E][d][F] (bit patterns); other arguments as in
+ * oracle_moe_forward.  Returns 0, or -1 on bad arguments. */
+int oracle_moe_forward_bf16w(const uint16_t* x, int64_t T, int64_t d, int64_t F, int E, int K, const float* wr,
+                             const float* bias, const uint16_t* w1, const uint16_t* w3, const uint16_t* w2,
+                             const int64_t* tokens, int64_t n_tokens, double* y, int32_t* ids, double* wts,
+                             double* h_out, int threads) {
+    if (!x || !wr || !w1 || !w3 || !w2 || !y) return -1;
+    if (T < 0 || d <= 0 || F <= 0 || E < 1 || E > 64 || K < 1 || K > E || n_tokens < 0) return -1;
+    if (tokens) {
+        for (int64_t n = 0; n < n_tokens; ++n)
+            if (tokens[n] < 0 || tokens[n] >= T) return -1;
+    } else if (n_tokens > T) {
+        return -1;
+    }
+    fwdb_ctx c = {x, d, F, E, K, wr, bias, w1, w3, w2, tokens, y, ids, wts, h_out};
+    parallel_for(n_tokens, threads, forward_bf16w_range, &c);
     return 0;
 }
 

@@ -289,4 +289,33 @@ def pin_forward_token_subset_and_expert_permutation(orc):
     assert np.allclose(outp["y"], full, rtol=1e-13, atol=1e-16)
 
 
+# ---------------------------------------------------------- bf16-weight layer
+
+
+def pin_bf16w_equals_int8_when_weights_are_codes_times_pow2(orc):
+    # bf16 weights w = q * 2^k are exact; with scales 2^k the int8 layer computes the same products
+    rng = np.random.default_rng(21)
+    L = tiny_layer(rng, T=6, d=32, F=40)
+    for key, sk in (("q1", "s1"), ("q3", "s3"), ("q2", "s2")):
+        L[sk] = np.full_like(L[sk], np.float32(2.0 ** -9))
+    w = {key: bf16_bits(L[key].astype(np.float32) * np.float32(2.0 ** -9)) for key in ("q1", "q3", "q2")}
+    a = fwd(orc, L, want_hidden=True)
+    b = orc.moe_forward_bf16w(L["x"], L["wr"], None, w["q1"], w["q3"], w["q2"], want_hidden=True)
+    assert np.array_equal(a["ids"], b["ids"]) and np.array_equal(a["h"], b["h"]) and np.array_equal(a["y"], b["y"])
+
+
+def pin_bf16w_identical_experts_is_dense_mlp(orc):
+    rng = np.random.default_rng(22)
+    T, d, F = 5, 24, 36
+    x = random_bf16(rng, (T, d), 1.0)
+    wr = (rng.standard_normal((2, d)) * 0.3).astype(np.float32)
+    w1, w3 = random_bf16(rng, (F, d), 0.05), random_bf16(rng, (F, d), 0.05)
+    w2 = random_bf16(rng, (d, F), 0.05)
+    rep = lambda a: np.ascontiguousarray(np.repeat(a[None], 2, axis=0))  # noqa: E731
+    out = orc.moe_forward_bf16w(x, wr, None, rep(w1), rep(w3), rep(w2))
+    f = synth.bf16_bits_to_f32
+    y_ref, _ = swiglu_torch(f(x), f(w1), f(w3), f(w2))
+    assert np.allclose(out["y"], y_ref, rtol=1e-12, atol=1e-15)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -25,6 +25,9 @@ MUTANTS = {
     "bias_sign": ("acc += (double)bias[e];", "acc -= (double)bias[e];"),
     "softmax_unnormalised": ("p[e] /= denom;", "(void)denom;"),
     "dropped_gate_weight": ("yt[i] += wts[k] * o[i];", "yt[i] += o[i];"),
+    "bf16w_down_transposed": ("acc += (double)bf16_value(r2[j]) * h[j];",
+                              "acc += (double)bf16_value(w2[j * d + i]) * h[j];"),
+    "bf16w_up_uses_gate": ("a3 += (double)bf16_value(r3[i]) * xd[i];", "a3 += (double)bf16_value(r1[i]) * xd[i];"),
     "router_ignores_last_input": ("for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i])",
                                   "for (int64_t i = 0; i + 1 < d; ++i) acc += (double)bf16_value(x[i])"),
 }
