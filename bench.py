@@ -40,6 +40,8 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
+    ap.add_argument("--weights", default="int8", choices=["int8", "bf16"],
+                    help="int8: ExpertsInt8 (the method); bf16: the unquantized comparator layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
@@ -59,14 +61,16 @@ def load_peaks():
 
 
 # ------------------------------------------------------------------ algorithmic work per launch
-def algorithmic(kind, wl, T, touched, rows_padded):
+def algorithmic(kind, wl, T, touched, rows_padded, wbytes=1):
     """Bytes (HBM-bound kernels) or FLOPs (tensor-bound kernels) one launch must move / do.
-    touched = experts with >= 1 token; rows_padded = permuted rows incl. per-expert padding."""
+    touched = experts with >= 1 token; rows_padded = permuted rows incl. per-expert padding;
+    wbytes = bytes per weight (1: int8 codes, plus 4-byte scales per row; 2: bf16, no scales)."""
     d, F, TK = wl.d, wl.F, T * wl.K
+    sc = 4 if wbytes == 1 else 0
     if kind == "gemv13":
-        return "bytes", touched * (2 * F * d + 2 * F * 4) + TK * d * 2 + TK * F * 2
+        return "bytes", touched * (2 * F * d * wbytes + 2 * F * sc) + TK * d * 2 + TK * F * 2
     if kind == "gemv2":
-        return "bytes", touched * (d * F + d * 4) + TK * F * 2 + TK * d * 4 + TK * 4 * 2
+        return "bytes", touched * (d * F * wbytes + d * sc) + TK * F * 2 + TK * d * 4 + TK * 4 * 2
     if kind == "gemm13":
         return "flops", 2.0 * TK * d * (2 * F)
     if kind == "gemm2":
@@ -305,21 +309,28 @@ def run_ours(args):
     wr = torch.from_numpy(synth.gen_router(wl)).to(dev)
     bias_np = synth.gen_bias(wl)
     bias = None if bias_np is None else torch.from_numpy(bias_np).to(dev)
-    Q, S = {}, {}
+    int8w = args.weights == "int8"
+    wbytes = 1 if int8w else 2
+    Q, S, Wb = {}, {}, {}
     q_ms = 0.0
-    qe0, qe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    jm.jamba_moe_timing_start(3 * E)  # the quantize launches, timed by the library's own events
     for which in ("w1", "w3", "w2"):
         rows, cols = synth.weight_shape(wl, which)
-        Q[which] = torch.empty((E, rows, cols), dtype=torch.int8, device=dev)
-        S[which] = torch.empty((E, rows), dtype=torch.float32, device=dev)
+        if int8w:
+            Q[which] = torch.empty((E, rows, cols), dtype=torch.int8, device=dev)
+            S[which] = torch.empty((E, rows), dtype=torch.float32, device=dev)
+        else:
+            Wb[which] = torch.empty((E, rows, cols), dtype=torch.bfloat16, device=dev)
         for e in range(E):
             w = to_dev(synth.gen_expert(wl, which, e))
-            qe0.record()
-            jm.jamba_moe_quantize(w, out=(Q[which][e], S[which][e]))
-            qe1.record()
-            torch.cuda.synchronize()
-            q_ms += qe0.elapsed_time(qe1)
+            if int8w:
+                jm.jamba_moe_quantize(w, out=(Q[which][e], S[which][e]))
+            else:
+                Wb[which][e].copy_(w)
             del w
+    torch.cuda.synchronize()
+    q_ms = jm.jamba_moe_timing_collect().get("quantize", (0.0, 0))[0]
+    jm.jamba_moe_timing_start(0)
     q_bytes = algorithmic("quantize", wl, T, 0, 0)[1]
     ws = torch.empty(jm.jamba_moe_workspace_size(T, d, F), dtype=torch.uint8, device=dev)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
@@ -327,9 +338,16 @@ def run_ours(args):
     tw = torch.empty((T, 2), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    def forward(xin):
+        if int8w:
+            jm.jamba_moe_forward(xin, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
+                                 topk_ids=ids, topk_w=tw, workspace=ws, path=path)
+        else:
+            jm.jamba_moe_forward_bf16w(xin, wr, bias, Wb["w1"], Wb["w3"], Wb["w2"], y=y, topk_ids=ids, topk_w=tw,
+                                       workspace=ws, path=path)
+
     def step():
-        jm.jamba_moe_forward(x, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y, topk_ids=ids,
-                             topk_w=tw, workspace=ws, path=path)
+        forward(x)
 
     def barrier():
         if world > 1:
@@ -369,8 +387,7 @@ def run_ours(args):
 
     def step_e2e():
         x_dev.copy_(x_host, non_blocking=True)
-        jm.jamba_moe_forward(x_dev, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
-                             topk_ids=ids, topk_w=tw, workspace=ws, path=path)
+        forward(x_dev)
         y_host.copy_(y, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -388,7 +405,7 @@ def run_ours(args):
     # ---- roofline of the dominant kernel
     dom = max(kernels, key=lambda k: kernels[k][0])
     dom_ms, dom_n = kernels[dom]
-    unit_kind, work = algorithmic(dom, wl, T, touched, rows_padded)
+    unit_kind, work = algorithmic(dom, wl, T, touched, rows_padded, wbytes)
     avg_s = dom_ms / dom_n / 1e3
     if unit_kind == "bytes":
         achieved, peak, unit, bound = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
@@ -399,13 +416,13 @@ def run_ours(args):
                 "peak_source": peaks["source"]}
     per_kernel = {}
     for k, (kms, n) in sorted(kernels.items(), key=lambda kv: -kv[1][0]):
-        uk, wk = algorithmic(k, wl, T, touched, rows_padded)
+        uk, wk = algorithmic(k, wl, T, touched, rows_padded, wbytes)
         a = wk / (kms / n / 1e3)
         per_kernel[k] = {"launches": n, "avg_us": kms / n * 1e3,
                          ("GB/s" if uk == "bytes" else "TFLOP/s"): a / (1e9 if uk == "bytes" else 1e12)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and int8w:
         setup = oracle_setup(wl, seed_x)
         rate, cores, n, dt = oracle_rate(wl, setup, args.cpu_budget_s)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
@@ -416,15 +433,17 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu"),
+            "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
+                           weights=("int8 codes + fp32 per-output-channel scales" if int8w
+                                    else "bf16 (unquantized comparator)")),
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 2},
             "gpu_launches": int(sum(n for _, n in kernels.values())),
             "clocks": clk.summary(), "kernels": per_kernel, "device_status": status,
             "routing": {"touched_experts": touched, "max_tokens_per_expert": int(counts.max())},
-            "quantize": {"ms": q_ms, "GB/s": q_bytes / (q_ms / 1e3) / 1e9,
-                         "frac_of_hbm": q_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"]},
+            "quantize": ({"ms": q_ms, "GB/s": q_bytes / (q_ms / 1e3) / 1e9,
+                          "frac_of_hbm": q_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"]} if q_ms > 0 else None),
         }
         print(json.dumps(out), flush=True)
     if world > 1:

@@ -122,6 +122,20 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
                            size_t workspace_bytes, void* stream, int path);
 
 /*
+ * jamba_moe_forward_bf16w — the same layer with unquantized bf16 expert weights (no ExpertsInt8):
+ * W1, W3 bf16 [n_experts][ffn][d], W2 bf16 [n_experts][d][ffn]; everything else as in
+ * jamba_moe_forward_path (same workspace size, same paths, same numerics minus the scales).  It
+ * is the comparator the Jamba-1.5 paper measures ExpertsInt8 against (§3.1 reports ExpertsInt8 at
+ * no extra latency, even slightly faster, than BF16 weights): here the decode path streams twice
+ * the weight bytes, and the prefill path loads the weight tiles straight into the MMA's layout
+ * without conversion.
+ */
+int jamba_moe_forward_bf16w(const uint16_t* x, const float* router_W, const float* router_bias,
+                            const uint16_t* W1, const uint16_t* W3, const uint16_t* W2, int64_t T, int64_t d,
+                            int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w,
+                            void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/*
  * jamba_moe_read_device_status — synchronises `stream`, then returns the status word the
  * kernels of the last forward call on `workspace` left there: JMOE_OK, JMOE_DEV_TIMEOUT (a
  * pipeline wait ran out of its bounded number of polls; the kernel released its resources and

@@ -65,6 +65,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_noalloc_scratch_capacity.argtypes = []
     lib.jamba_moe_noalloc_scratch_needed.restype = sz
     lib.jamba_moe_noalloc_scratch_needed.argtypes = [i64, i64, i64]
+    lib.jamba_moe_forward_bf16w.restype = c_int
+    lib.jamba_moe_forward_bf16w.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, sz,
+                                            vp, c_int]
     lib.jamba_moe_debug_skip_copy.restype = c_int
     lib.jamba_moe_debug_skip_copy.argtypes = [c_int]
     lib.jamba_moe_kernel_name.restype = ctypes.c_char_p
@@ -176,6 +179,45 @@ def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Opti
                                     workspace.data_ptr(), workspace.numel(), _stream_ptr(stream), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward")
+    return y, topk_ids, topk_w
+
+
+def jamba_moe_forward_bf16w(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor],
+                            W1: torch.Tensor, W3: torch.Tensor, W2: torch.Tensor, y: Optional[torch.Tensor] = None,
+                            topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                            path: int = PATH_AUTO):
+    """The same layer with unquantized bf16 expert weights W1, W3 [16][ffn][d], W2 [16][d][ffn]
+    (the BF16 comparator of ExpertsInt8).  Returns (y, topk_ids, topk_w)."""
+    lib = load_library()
+    _check(x, "x", torch.bfloat16)
+    T, d = x.shape
+    E, ffn = W1.shape[0], W1.shape[1]
+    _check(router_W, "router_W", torch.float32, (E, d))
+    if router_bias is not None:
+        _check(router_bias, "router_bias", torch.float32, (E,))
+    _check(W1, "W1", torch.bfloat16, (E, ffn, d))
+    _check(W3, "W3", torch.bfloat16, (E, ffn, d))
+    _check(W2, "W2", torch.bfloat16, (E, d, ffn))
+    y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device) if y is None else y
+    topk_ids = torch.empty((T, TOP_K), dtype=torch.int32, device=x.device) if topk_ids is None else topk_ids
+    topk_w = torch.empty((T, TOP_K), dtype=torch.float32, device=x.device) if topk_w is None else topk_w
+    _check(y, "y", torch.bfloat16, (T, d))
+    _check(topk_ids, "topk_ids", torch.int32, (T, TOP_K))
+    _check(topk_w, "topk_w", torch.float32, (T, TOP_K))
+    need = jamba_moe_workspace_size(T, d, ffn, E, TOP_K)
+    if need == 0:
+        raise JmoeError(2, "jamba_moe_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    st = lib.jamba_moe_forward_bf16w(x.data_ptr(), router_W.data_ptr(), p(router_bias), W1.data_ptr(), W3.data_ptr(),
+                                     W2.data_ptr(), T, d, ffn, E, TOP_K, y.data_ptr(), topk_ids.data_ptr(),
+                                     topk_w.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream),
+                                     int(path))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_forward_bf16w")
     return y, topk_ids, topk_w
 
 

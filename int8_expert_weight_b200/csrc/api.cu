@@ -13,7 +13,17 @@ cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias,
 cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
                            cudaStream_t st);
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
-                          uint16_t* x_perm, cudaStream_t st, int num_sms);
+                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid);
+cudaError_t launch_gemv13_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const uint16_t* W1,
+                                const uint16_t* W3, uint16_t* h, int64_t T, int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemv2_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const uint16_t* W2,
+                               const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemm13_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const uint16_t* W1,
+                                const uint16_t* W3, uint16_t* h, int64_t rows_cap, int64_t d, int64_t F,
+                                cudaStream_t st);
+cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const uint16_t* W2,
+                               const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F,
+                               cudaStream_t st);
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
                           int64_t F, cudaStream_t st);
@@ -135,15 +145,20 @@ size_t jamba_moe_workspace_size(int64_t T, int64_t d, int64_t ffn, int n_experts
     return make_layout(T, d, ffn).total;
 }
 
-int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
-                           const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,
-                           int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y,
-                           int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream,
-                           int path) {
-    if (!x || !router_W || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
+}  // extern "C"
+
+namespace {
+
+// The layer with either int8 weights (codes + per-row scales, w8) or unquantized bf16 weights.
+int forward_impl(const uint16_t* x, const float* router_W, const float* router_bias, const void* W1,
+                 const float* S1, const void* W3, const float* S3, const void* W2, const float* S2, bool w8,
+                 int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids,
+                 float* topk_w, void* workspace, size_t workspace_bytes, void* stream, int path) {
+    if (!x || !router_W || !W1 || !W3 || !W2 || !y || !workspace) return JMOE_ERR_NULL;
+    if (w8 && (!S1 || !S3 || !S2)) return JMOE_ERR_NULL;
     if (!shape_ok(T, d, ffn, n_experts, top_k)) return JMOE_ERR_SHAPE;
     if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
-    const void* ptrs16[] = {x, Q1, Q3, Q2, y, router_W};
+    const void* ptrs16[] = {x, W1, W3, W2, y, router_W};
     for (const void* p : ptrs16)
         if (!aligned16(p)) return JMOE_ERR_ALIGN;
     const void* ptrs4[] = {router_bias, S1, S3, S2, topk_ids, topk_w};
@@ -166,6 +181,12 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
     const int sms = num_sms_current();
     // Few tokens per expert: stream the weights (GEMV); otherwise grouped tensor-core GEMMs.
     if (path == JMOE_PATH_AUTO) path = (T <= kGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
+    const int8_t* Q1 = static_cast<const int8_t*>(W1);
+    const int8_t* Q3 = static_cast<const int8_t*>(W3);
+    const int8_t* Q2 = static_cast<const int8_t*>(W2);
+    const uint16_t* B1 = static_cast<const uint16_t*>(W1);
+    const uint16_t* B3 = static_cast<const uint16_t*>(W3);
+    const uint16_t* B2 = static_cast<const uint16_t*>(W2);
 
     cudaError_t e;
     {
@@ -181,28 +202,32 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
     if (path == JMOE_PATH_GEMV) {
         {
             TimedLaunch t(JMOE_KERNEL_GEMV13, st);
-            e = launch_gemv13(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st);
+            e = w8 ? launch_gemv13(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st)
+                   : launch_gemv13_bf16w(hdr, perm, x, B1, B3, h, T, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
         {
             TimedLaunch t(JMOE_KERNEL_GEMV2, st);
-            e = launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st);
+            e = w8 ? launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st)
+                   : launch_gemv2_bf16w(hdr, perm, h, B2, wts, slots, T, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
     } else {
         {
             TimedLaunch t(JMOE_KERNEL_GATHER, st);
-            e = launch_gather(x, perm, hdr, d, L.rows_cap, x_perm, st, sms);
+            e = launch_gather(x, perm, hdr, d, L.rows_cap, x_perm, st, sms, w8);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
         {
             TimedLaunch t(JMOE_KERNEL_GEMM13, st);
-            e = launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st);
+            e = w8 ? launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st)
+                   : launch_gemm13_bf16w(hdr, perm, x_perm, B1, B3, h, L.rows_cap, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
         {
             TimedLaunch t(JMOE_KERNEL_GEMM2, st);
-            e = launch_gemm2(hdr, perm, h, Q2, S2, wts, slots, L.rows_cap, d, ffn, st);
+            e = w8 ? launch_gemm2(hdr, perm, h, Q2, S2, wts, slots, L.rows_cap, d, ffn, st)
+                   : launch_gemm2_bf16w(hdr, perm, h, B2, wts, slots, L.rows_cap, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
     }
@@ -211,6 +236,27 @@ int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float
         e = launch_combine(slots, T, d, y, st, sms);
     }
     return to_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
+                           const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,
+                           int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y,
+                           int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream,
+                           int path) {
+    return forward_impl(x, router_W, router_bias, Q1, S1, Q3, S3, Q2, S2, true, T, d, ffn, n_experts, top_k, y,
+                        topk_ids, topk_w, workspace, workspace_bytes, stream, path);
+}
+
+int jamba_moe_forward_bf16w(const uint16_t* x, const float* router_W, const float* router_bias, const uint16_t* W1,
+                            const uint16_t* W3, const uint16_t* W2, int64_t T, int64_t d, int64_t ffn, int n_experts,
+                            int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w, void* workspace,
+                            size_t workspace_bytes, void* stream, int path) {
+    return forward_impl(x, router_W, router_bias, W1, nullptr, W3, nullptr, W2, nullptr, false, T, d, ffn, n_experts,
+                        top_k, y, topk_ids, topk_w, workspace, workspace_bytes, stream, path);
 }
 
 int jamba_moe_forward(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,

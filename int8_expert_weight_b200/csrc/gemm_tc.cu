@@ -28,7 +28,6 @@ namespace jmoe {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kStages = 3;
 constexpr int kConvWarps = 8;
 constexpr int kEpiWarps = 4;
 constexpr int kGemmThreads = (2 + kConvWarps + kEpiWarps) * 32;
@@ -51,11 +50,15 @@ struct GemmArgs {
     int skip_copy;        // test hook: CTA 0 skips the copies of its second K step (a wait then runs out)
 };
 
-template <int BN>
+// Shared-memory ring: per stage the activation tile, the bf16 weight tile the MMA reads and, for
+// int8 weights, the int8 tile as loaded (converted into the bf16 tile by the converter warps).
+// Unquantized bf16 weights are loaded straight into the bf16 tile, which leaves room for 4 stages.
+template <int BN, bool kW8>
 struct StageLayout {
-    static constexpr int kA = kBM * kBK * 2;   // bf16 activations
-    static constexpr int kBbf = BN * kBK * 2;  // bf16 weights (converted)
-    static constexpr int kBq = BN * kBK;       // int8 weights (as loaded)
+    static constexpr int kStages = kW8 ? 3 : 4;
+    static constexpr int kA = kBM * kBK * 2;          // bf16 activations
+    static constexpr int kBbf = BN * kBK * 2;         // bf16 weights (converted or loaded)
+    static constexpr int kBq = kW8 ? BN * kBK : 0;    // int8 weights (as loaded)
     static constexpr int kStage = kA + kBbf + kBq;
     static constexpr int kSmem = kStages * kStage + 1024 + 256;
 };
@@ -109,11 +112,12 @@ __device__ __forceinline__ bool tile_coord(const WsHeader* hdr, const GemmArgs& 
     return false;
 }
 
-template <bool kDual, int BN>
+template <bool kDual, int BN, bool kW8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, GemmArgs p) {
-    using SL = StageLayout<BN>;
+    using SL = StageLayout<BN, kW8>;
+    constexpr int kStages = SL::kStages;
     static_assert(!kDual || BN == 256, "the SwiGLU tile pairs 128 gate rows with 128 up rows");
     constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
     extern __shared__ uint8_t smem_raw[];
@@ -163,9 +167,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tc::tc_fence_after();
     const uint32_t tmem = tmem_holder;
     const int KB = p.K / kBK;
-    constexpr uint32_t kTxBytes = SL::kA + SL::kBq;
+    constexpr uint32_t kTxBytes = SL::kA + (kW8 ? SL::kBq : SL::kBbf);
     constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, BN);
-    int issued_round[kStages] = {-1, -1, -1};  // producer: last round issued on each stage
+    int issued_round[kStages];  // producer: last round issued on each stage (-1: none)
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
     int mma_issued = 0;
 
     if (warp == 0) {
@@ -188,8 +194,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     if (p.skip_copy && blockIdx.x == 0 && L == (int)blockIdx.x && kb == 1) continue;
                     tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
                     tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
-                    tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
-                    if (kDual) tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                    if (kW8) {
+                        tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                        if (kDual)
+                            tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                    } else {  // bf16 weights land in the MMA's SWIZZLE_128B tile directly (128 bytes per row)
+                        tc::tma_load_2d(sBbf(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                        if (kDual)
+                            tc::tma_load_2d(sBbf(s) + (BN / 2) * 128, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                    }
                     issued_round[s] = r;
                 }
                 if (!ok) break;
@@ -211,7 +224,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages, r = g / kStages;
                     if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls) ||
-                        !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, p.max_polls)) {
+                        (kW8 && !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, p.max_polls))) {
                         if (!abort_flag) fail(p.hdr, &abort_flag);
                         ok = false;
                         break;
@@ -232,6 +245,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         __syncwarp();
     } else if (warp < 2 + kConvWarps) {
+        if (kW8) {  // bf16 weights need no conversion
         // ---------------- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte
         // chunk c of row r stored at chunk c ^ (r & 7) of the row's 128 bytes)
         const int t = threadIdx.x - 64;
@@ -267,6 +281,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             if (!ok) break;
         }
+        }
     } else {
         // ---------------- epilogue
         const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
@@ -298,21 +313,25 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     uint32_t packed[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
-                        const float g0 = __uint_as_float(a1[i]) * __ldg(s1 + c + i);
-                        const float g1 = __uint_as_float(a1[i + 1]) * __ldg(s1 + c + i + 1);
-                        const float u0 = __uint_as_float(a3[i]) * __ldg(s3 + c + i);
-                        const float u1 = __uint_as_float(a3[i + 1]) * __ldg(s3 + c + i + 1);
+                        const float g0 = __uint_as_float(a1[i]) * (kW8 ? __ldg(s1 + c + i) : 1.0f);
+                        const float g1 = __uint_as_float(a1[i + 1]) * (kW8 ? __ldg(s1 + c + i + 1) : 1.0f);
+                        const float u0 = __uint_as_float(a3[i]) * (kW8 ? __ldg(s3 + c + i) : 1.0f);
+                        const float u1 = __uint_as_float(a3[i + 1]) * (kW8 ? __ldg(s3 + c + i + 1) : 1.0f);
                         packed[i / 2] = (uint32_t)f32_to_bf16_bits(silu(g0) * u0) |
                                         ((uint32_t)f32_to_bf16_bits(silu(g1) * u1) << 16);
                     }
-                    // h feeds the down-projection GEMM as its activation operand: store every group of
-                    // 4 columns in the 0, 2, 1, 3 order that GEMM's weight conversion produces
+                    // h feeds the down-projection GEMM as its activation operand: with int8 weights,
+                    // store every group of 4 columns in the 0, 2, 1, 3 order the weight conversion produces
                     uint4* dst = reinterpret_cast<uint4*>(hrow + c);
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
-                        const uint2 a = swap_mid4(packed[4 * v], packed[4 * v + 1]);
-                        const uint2 b = swap_mid4(packed[4 * v + 2], packed[4 * v + 3]);
-                        dst[v] = make_uint4(a.x, a.y, b.x, b.y);
+                        if (kW8) {
+                            const uint2 a = swap_mid4(packed[4 * v], packed[4 * v + 1]);
+                            const uint2 b = swap_mid4(packed[4 * v + 2], packed[4 * v + 3]);
+                            dst[v] = make_uint4(a.x, a.y, b.x, b.y);
+                        } else {
+                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                        }
                     }
                 }
             } else {
@@ -331,10 +350,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             float4 o;
-                            o.x = wt * (__ldg(s2 + c + 4 * k + 0) * __uint_as_float(v[4 * k + 0]));
-                            o.y = wt * (__ldg(s2 + c + 4 * k + 1) * __uint_as_float(v[4 * k + 1]));
-                            o.z = wt * (__ldg(s2 + c + 4 * k + 2) * __uint_as_float(v[4 * k + 2]));
-                            o.w = wt * (__ldg(s2 + c + 4 * k + 3) * __uint_as_float(v[4 * k + 3]));
+                            o.x = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
+                            o.y = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
+                            o.z = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
+                            o.w = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
                             dst[k] = o;
                         }
                     }
@@ -413,11 +432,11 @@ int band_for(int K) {
     return b < 1 ? 1 : (b > 16 ? 16 : b);
 }
 
-template <bool kDual, int BN>
+template <bool kDual, int BN, bool kW8>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const GemmArgs& p,
                           int64_t m_tiles_cap, cudaStream_t st) {
-    using SL = StageLayout<BN>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    using SL = StageLayout<BN, kW8>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN, kW8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SL::kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (fewer when there are fewer tile slots)
@@ -429,7 +448,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
     }
     int64_t grid = m_tiles_cap * p.n_tiles;
     if (grid > sms) grid = sms;
-    return launch_pdl(gemm_tc_kernel<kDual, BN>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta, tb0,
+    return launch_pdl(gemm_tc_kernel<kDual, BN, kW8>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta, tb0,
                       tb1, p);
 }
 
@@ -451,7 +470,7 @@ cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_
                nullptr,      h,             nullptr,     (int)d,
                (int)F,       (int)(F / 128), band_for((int)d), g_skip_copy ? kTestMaxPolls : kMaxPolls,
                g_skip_copy};
-    return launch_gemm_t<true, 256>(ta, tb0, tb1, p, rows_cap / kBM, st);
+    return launch_gemm_t<true, 256, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
 // out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment.
@@ -467,8 +486,45 @@ cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, 
                wts,         nullptr,      out_slot,    (int)F,
                (int)d,      (int)(d / BN), band_for((int)F), g_skip_copy ? kTestMaxPolls : kMaxPolls,
                0};
-    if (BN == 256) return launch_gemm_t<false, 256>(ta, tb0, tb0, p, rows_cap / kBM, st);
-    return launch_gemm_t<false, 128>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    if (BN == 256) return launch_gemm_t<false, 256, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    return launch_gemm_t<false, 128, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
+}
+
+// The same two GEMMs with unquantized bf16 weights: the weight tiles are TMA-loaded in the
+// MMA's layout, nothing is converted, no scales are applied, and activations keep their k order.
+cudaError_t launch_gemm13_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const uint16_t* W1,
+                                const uint16_t* W3, uint16_t* h, int64_t rows_cap, int64_t d, int64_t F,
+                                cudaStream_t st) {
+    CUtensorMap ta, tb0, tb1;
+    if (!make_map(&ta, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kBM, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, W1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)kExperts * F, d, 128, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb1, W3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)kExperts * F, d, 128, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr,          perm,          nullptr,     nullptr,
+               nullptr,      h,             nullptr,     (int)d,
+               (int)F,       (int)(F / 128), band_for((int)d), kMaxPolls,
+               0};
+    return launch_gemm_t<true, 256, false>(ta, tb0, tb1, p, rows_cap / kBM, st);
+}
+
+cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const uint16_t* W2,
+                               const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F,
+                               cudaStream_t st) {
+    const int BN = (d % 256 == 0) ? 256 : 128;
+    CUtensorMap ta, tb0;
+    if (!make_map(&ta, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, W2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)kExperts * d, F, BN, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr,         perm,         nullptr,     nullptr,
+               wts,         nullptr,      out_slot,    (int)F,
+               (int)d,      (int)(d / BN), band_for((int)F), kMaxPolls,
+               0};
+    if (BN == 256) return launch_gemm_t<false, 256, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    return launch_gemm_t<false, 128, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
 
 }  // namespace jmoe

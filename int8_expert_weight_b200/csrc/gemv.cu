@@ -26,9 +26,9 @@ struct GemvArgs {
     const WsHeader* hdr;
     const int32_t* perm;   // [rows] assignment index (t*K + k) of each permuted row, -1 = padding
     const uint16_t* act;   // gemv13: x [T][d]; gemv2: h [rows][F]
-    const int8_t* qa;      // gemv13: Q1 [E][F][d]; gemv2: Q2 [E][d][F]
-    const int8_t* qb;      // gemv13: Q3 [E][F][d]; gemv2: unused
-    const float* sa;       // S1 [E][F] / S2 [E][d]
+    const void* qa;        // gemv13: W1 [E][F][d]; gemv2: W2 [E][d][F] (int8 codes, or bf16 weights)
+    const void* qb;        // gemv13: W3 [E][F][d]; gemv2: unused
+    const float* sa;       // S1 [E][F] / S2 [E][d] (int8 codes only)
     const float* sb;       // S3 [E][F]
     const float* wts;      // gemv2: routing weight of each assignment [T*K]
     uint16_t* h_out;       // gemv13: h [rows][F]
@@ -37,41 +37,72 @@ struct GemvArgs {
     int64_t N;             // weight rows per expert: F (gemv13) or d (gemv2)
 };
 
-template <bool kDual>
+// One k-step (16 consecutive k per lane) of weights for rows g and g+8: int8 codes fill one
+// 16-byte vector per row, bf16 weights two.
+template <bool kDual, bool kW8>
 struct WeightRegs {
-    uint4 a0, a1, b0, b1;  // rows g and g+8 of matrix a (and b)
+    static constexpr int kV = kW8 ? 1 : 2;
+    uint4 a0[kV], a1[kV], b0[kV], b1[kV];  // rows g and g+8 of matrix a (and b)
 };
 
 __device__ __forceinline__ uint32_t word(const uint4& v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
+// Word m (0..7) of 16 consecutive bf16 values held in two vectors.
+__device__ __forceinline__ uint32_t word8(const uint4 (&v)[2], int m) { return word(v[m >> 2], m & 3); }
+__device__ __forceinline__ uint32_t word8(const uint4 (&v)[1], int m) { return word(v[0], m & 3); }
 
-template <int NT, bool kDual>
-__device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[NT][4], const WeightRegs<kDual>& w,
-                                         const uint4 (&xa)[NT][2], const S8Consts& k) {
+template <int NT, bool kDual, bool kW8>
+__device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[NT][4],
+                                         const WeightRegs<kDual, kW8>& w, const uint4 (&xa)[NT][2],
+                                         const S8Consts& k) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        // A fragment: k positions (2c, 2c+1) <- bytes 4j, 4j+2; (2c+8, 2c+9) <- bytes 4j+1, 4j+3.
-        const uint32_t wa0 = word(w.a0, j), wa1 = word(w.a1, j);
-        const uint32_t a0 = s8x2_even_to_bf16x2(wa0, k), a1 = s8x2_even_to_bf16x2(wa1, k);
-        const uint32_t a2 = s8x2_odd_to_bf16x2(wa0, k), a3 = s8x2_odd_to_bf16x2(wa1, k);
+        uint32_t a0, a1, a2, a3, c0 = 0, c1 = 0, c2 = 0, c3 = 0;
         uint32_t b0[NT], b1[NT];
+        if (kW8) {
+            // A fragment: k positions (2c, 2c+1) <- bytes 4j, 4j+2; (2c+8, 2c+9) <- bytes 4j+1, 4j+3.
+            const uint32_t wa0 = word(w.a0[0], j), wa1 = word(w.a1[0], j);
+            a0 = s8x2_even_to_bf16x2(wa0, k);
+            a1 = s8x2_even_to_bf16x2(wa1, k);
+            a2 = s8x2_odd_to_bf16x2(wa0, k);
+            a3 = s8x2_odd_to_bf16x2(wa1, k);
+            if (kDual) {
+                const uint32_t wb0 = word(w.b0[0], j), wb1 = word(w.b1[0], j);
+                c0 = s8x2_even_to_bf16x2(wb0, k);
+                c1 = s8x2_even_to_bf16x2(wb1, k);
+                c2 = s8x2_odd_to_bf16x2(wb0, k);
+                c3 = s8x2_odd_to_bf16x2(wb1, k);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                // activations 4j..4j+3 of this lane's 16: words 2j = (4j, 4j+1), 2j+1 = (4j+2, 4j+3)
+                const uint32_t lo = word8(xa[nt], 2 * j), hi = word8(xa[nt], 2 * j + 1);
+                b0[nt] = pair_lo(lo, hi);
+                b1[nt] = pair_hi(lo, hi);
+            }
+        } else {
+            // bf16 weights: k positions (2c, 2c+1) <- elements 4j, 4j+1; (2c+8, 2c+9) <- 4j+2, 4j+3
+            a0 = word8(w.a0, 2 * j);
+            a2 = word8(w.a0, 2 * j + 1);
+            a1 = word8(w.a1, 2 * j);
+            a3 = word8(w.a1, 2 * j + 1);
+            if (kDual) {
+                c0 = word8(w.b0, 2 * j);
+                c2 = word8(w.b0, 2 * j + 1);
+                c1 = word8(w.b1, 2 * j);
+                c3 = word8(w.b1, 2 * j + 1);
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                b0[nt] = word8(xa[nt], 2 * j);
+                b1[nt] = word8(xa[nt], 2 * j + 1);
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            // activations 4j..4j+3 of this lane's 16: words 2j = (4j, 4j+1), 2j+1 = (4j+2, 4j+3)
-            const uint4& v = xa[nt][j >> 1];
-            const uint32_t lo = (j & 1) ? v.z : v.x;
-            const uint32_t hi = (j & 1) ? v.w : v.y;
-            b0[nt] = pair_lo(lo, hi);
-            b1[nt] = pair_hi(lo, hi);
             mma_bf16_16816(acc_a[nt], a0, a1, a2, a3, b0[nt], b1[nt]);
-        }
-        if (kDual) {
-            const uint32_t wb0 = word(w.b0, j), wb1 = word(w.b1, j);
-            const uint32_t c0 = s8x2_even_to_bf16x2(wb0, k), c1 = s8x2_even_to_bf16x2(wb1, k);
-            const uint32_t c2 = s8x2_odd_to_bf16x2(wb0, k), c3 = s8x2_odd_to_bf16x2(wb1, k);
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(acc_b[nt], c0, c1, c2, c3, b0[nt], b1[nt]);
+            if (kDual) mma_bf16_16816(acc_b[nt], c0, c1, c2, c3, b0[nt], b1[nt]);
         }
     }
 }
@@ -82,17 +113,22 @@ __device__ __forceinline__ void mma_step(float (&acc_a)[NT][4], float (&acc_b)[N
 // pointer increment per batch; the U steps are immediate offsets from it.  Rows of tokens past the
 // expert's count point at a valid row: their MMA columns are computed and then ignored.
 // Returns the CTA-reduced accumulators in shared memory red[mat][nt][lane*4 + i].
-template <int NT, bool kDual, int U>
+template <int NT, bool kDual, bool kW8, int U>
 __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, const uint16_t* const (&rows)[NT],
                                           float* red /* [kGemvWarps][2][NT][128] */) {
+    using W = WeightRegs<kDual, kW8>;
+    constexpr int kEl = kW8 ? 1 : 2;  // bytes per weight
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
     const int64_t K = p.K;
-    constexpr int kStride = kGemvWarps * 64;  // bytes (int8) / elements (bf16) between a warp's steps
-    const int8_t* pa0 = p.qa + ((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64;
-    const int8_t* pa1 = pa0 + 8 * K;
-    const int8_t* pb0 = kDual ? p.qb + ((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64 : nullptr;
-    const int8_t* pb1 = kDual ? pb0 + 8 * K : nullptr;
+    constexpr int kStride = kGemvWarps * 64;  // elements between a warp's steps
+    const uint8_t* pa0 =
+        static_cast<const uint8_t*>(p.qa) + (((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64) * kEl;
+    const uint8_t* pa1 = pa0 + 8 * K * kEl;
+    const uint8_t* pb0 =
+        kDual ? static_cast<const uint8_t*>(p.qb) + (((int64_t)e * p.N + j0 + g) * K + 16 * c + warp * 64) * kEl
+              : nullptr;
+    const uint8_t* pb1 = kDual ? pb0 + 8 * K * kEl : nullptr;
     const uint16_t* px[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) px[nt] = rows[nt] + 16 * c + warp * 64;
@@ -106,16 +142,19 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
     const int steps = (int)(K / 64);
     const S8Consts k = s8_consts();
     for (int s0 = warp; s0 < steps; s0 += kGemvWarps * U) {
-        WeightRegs<kDual> w[U];
+        W w[U];
         uint4 xa[U][NT][2];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             if (s0 + u * kGemvWarps < steps) {
-                w[u].a0 = ld_stream_v4(pa0 + u * kStride);
-                w[u].a1 = ld_stream_v4(pa1 + u * kStride);
-                if (kDual) {
-                    w[u].b0 = ld_stream_v4(pb0 + u * kStride);
-                    w[u].b1 = ld_stream_v4(pb1 + u * kStride);
+#pragma unroll
+                for (int v = 0; v < W::kV; ++v) {
+                    w[u].a0[v] = ld_stream_v4(pa0 + u * kStride * kEl + 16 * v);
+                    w[u].a1[v] = ld_stream_v4(pa1 + u * kStride * kEl + 16 * v);
+                    if (kDual) {
+                        w[u].b0[v] = ld_stream_v4(pb0 + u * kStride * kEl + 16 * v);
+                        w[u].b1[v] = ld_stream_v4(pb1 + u * kStride * kEl + 16 * v);
+                    }
                 }
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
@@ -126,12 +165,12 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (s0 + u * kGemvWarps < steps) mma_step<NT, kDual>(acc_a, acc_b, w[u], xa[u], k);
-        pa0 += U * kStride;
-        pa1 += U * kStride;
+            if (s0 + u * kGemvWarps < steps) mma_step<NT, kDual, kW8>(acc_a, acc_b, w[u], xa[u], k);
+        pa0 += U * kStride * kEl;
+        pa1 += U * kStride * kEl;
         if (kDual) {
-            pb0 += U * kStride;
-            pb1 += U * kStride;
+            pb0 += U * kStride * kEl;
+            pb1 += U * kStride * kEl;
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) px[nt] += U * kStride;
@@ -156,8 +195,10 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
     __syncthreads();
 }
 
-template <int NT, bool kDual>
-__global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? 2 : 1)) gemv_kernel(GemvArgs p) {
+template <int NT, bool kDual, bool kW8>
+__global__ void __launch_bounds__(kGemvWarps * 32,
+                                  kW8 ? ((NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? 2 : 1)) : ((NT == 1) ? 2 : 1))
+    gemv_kernel(GemvArgs p) {
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
     pdl_wait();
     const WsHeader* hdr = p.hdr;
@@ -181,7 +222,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4)
                 rows[nt] = p.act + (row0 + nn) * p.K;
             }
         }
-        gemv_pass<NT, kDual, 2>(p, e, j0, rows, red);
+        gemv_pass<NT, kDual, kW8, 2>(p, e, j0, rows, red);
         pdl_trigger();  // main loop done: the next kernel may start launching
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
@@ -192,12 +233,13 @@ __global__ void __launch_bounds__(kGemvWarps * 32, (NT == 1) ? ((kDual) ? 3 : 4)
             if (n >= m) continue;
             const int64_t jr = j0 + row;
             if (kDual) {
-                const float a1 = red[o] * p.sa[(int64_t)e * p.N + jr];
-                const float a3 = red[NT * 128 + o] * p.sb[(int64_t)e * p.N + jr];
+                const float a1 = kW8 ? red[o] * p.sa[(int64_t)e * p.N + jr] : red[o];
+                const float a3 = kW8 ? red[NT * 128 + o] * p.sb[(int64_t)e * p.N + jr] : red[NT * 128 + o];
                 p.h_out[(row0 + n) * p.N + jr] = f32_to_bf16_bits(silu(a1) * a3);
             } else {
                 const int32_t a = p.perm[row0 + n];
-                p.slot_out[(int64_t)a * p.N + jr] = p.wts[a] * (p.sa[(int64_t)e * p.N + jr] * red[o]);
+                const float v = kW8 ? p.sa[(int64_t)e * p.N + jr] * red[o] : red[o];
+                p.slot_out[(int64_t)a * p.N + jr] = p.wts[a] * v;
             }
         }
         __syncthreads();  // red is reused by the next pass
@@ -209,26 +251,39 @@ static int gemv_nt(int64_t T) {
     return avg <= 6 ? 1 : (avg <= 12 ? 2 : 4);
 }
 
-template <bool kDual>
+template <bool kDual, bool kW8>
 static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st) {
     dim3 grid((unsigned)(p.N / kGemvRows), kExperts);
-    if (nt == 1) return launch_pdl(gemv_kernel<1, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
-    if (nt == 2) return launch_pdl(gemv_kernel<2, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
-    return launch_pdl(gemv_kernel<4, kDual>, grid, dim3(kGemvWarps * 32), 0, st, p);
+    if (nt == 1) return launch_pdl(gemv_kernel<1, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
+    if (nt == 2) return launch_pdl(gemv_kernel<2, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
+    return launch_pdl(gemv_kernel<4, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
 }
 
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
                           int64_t F, cudaStream_t st) {
     GemvArgs p{hdr, perm, x, Q1, Q3, S1, S3, nullptr, h, nullptr, d, F};
-    return launch_gemv_t<true>(p, gemv_nt(T), st);
+    return launch_gemv_t<true, true>(p, gemv_nt(T), st);
 }
 
 cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
                          const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
                          cudaStream_t st) {
     GemvArgs p{hdr, perm, h, Q2, nullptr, S2, nullptr, wts, nullptr, out_slot, F, d};
-    return launch_gemv_t<false>(p, gemv_nt(T), st);
+    return launch_gemv_t<false, true>(p, gemv_nt(T), st);
+}
+
+// The same two kernels with unquantized bf16 weights (no dequantization, no scales).
+cudaError_t launch_gemv13_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const uint16_t* W1,
+                                const uint16_t* W3, uint16_t* h, int64_t T, int64_t d, int64_t F, cudaStream_t st) {
+    GemvArgs p{hdr, perm, x, W1, W3, nullptr, nullptr, nullptr, h, nullptr, d, F};
+    return launch_gemv_t<true, false>(p, gemv_nt(T), st);
+}
+
+cudaError_t launch_gemv2_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const uint16_t* W2,
+                               const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F, cudaStream_t st) {
+    GemvArgs p{hdr, perm, h, W2, nullptr, nullptr, nullptr, wts, nullptr, out_slot, F, d};
+    return launch_gemv_t<false, false>(p, gemv_nt(T), st);
 }
 
 }  // namespace jmoe

@@ -96,13 +96,14 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
         for (int r = seg[e] + hist[e] + tid; r < seg[e + 1]; r += kPermThreads) perm[r] = -1;
 }
 
-// x_perm[r] = x[perm[r] / K] for real rows (elements 1 and 2 of every group of 4 swapped, the k
-// order of the tensor-core path), zeros for padding rows; rows past the last segment are left
-// alone.  16-byte vector copies, one warp per row.
+// x_perm[r] = x[perm[r] / K] for real rows (with `swap`, elements 1 and 2 of every group of 4
+// swapped: the k order of the int8 tensor-core path), zeros for padding rows; rows past the last
+// segment are left alone.  16-byte vector copies, one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ perm,
                                                           const WsHeader* __restrict__ hdr, int64_t d,
-                                                          int64_t cap_rows, uint16_t* __restrict__ x_perm) {
+                                                          int64_t cap_rows, uint16_t* __restrict__ x_perm,
+                                                          int swap) {
     const int lane = threadIdx.x & 31;
     pdl_wait();
     pdl_trigger();
@@ -114,12 +115,14 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         if (a < 0) {
             for (int64_t c = lane; c < chunks; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
         } else {
-            // elements 1 and 2 of every group of 4 swapped: the k order of the GEMM path's weights
+            // with int8 weights, elements 1 and 2 of every group of 4 swapped: the k order of the
+            // converted weight tiles
             const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(a / kTopK) * d);
             for (int64_t c = lane; c < chunks; c += 32) {
                 const uint4 v = ld_nc_v4(src + c);
-                dst[c] = make_uint4(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632),
-                                    __byte_perm(v.z, v.w, 0x5410), __byte_perm(v.z, v.w, 0x7632));
+                dst[c] = swap ? make_uint4(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632),
+                                           __byte_perm(v.z, v.w, 0x5410), __byte_perm(v.z, v.w, 0x7632))
+                              : v;
             }
         }
     }
@@ -131,12 +134,12 @@ cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t
 }
 
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
-                          uint16_t* x_perm, cudaStream_t st, int num_sms) {
+                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid) {
     int64_t blocks = (cap_rows + 7) / 8;
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     if (blocks < 1) blocks = 1;
     return launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, perm, hdr, d, cap_rows,
-                      x_perm);
+                      x_perm, swap_mid ? 1 : 0);
 }
 
 }  // namespace jmoe
