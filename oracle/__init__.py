@@ -2,7 +2,8 @@
 
 ctypes wrapper around ``oracle.c``, the plain fp64 CPU implementation of the
 ExpertsInt8 mixture-of-experts layer (Jamba-1.5 paper, §3.1 "ExpertsInt8" and
-"Model Architecture").  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+"Model Architecture"), of the same layer with unquantized bf16 weights, and of the
+dense ExpertsInt8 MLP of the layers without MoE.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 CPU-baseline leg of ``bench.py`` may import this package.  It shares no code
 with the CUDA path (``int8_expert_weight_b200``), and the two never import
 each other; the only common dependency is the input generator ``synth``.
@@ -45,6 +46,8 @@ class Oracle:
         lib.oracle_moe_forward_bf16w.restype = c_int
         lib.oracle_moe_forward_bf16w.argtypes = [vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, vp, vp, i64, vp,
                                                  vp, vp, vp, c_int]
+        lib.oracle_mlp_forward.restype = c_int
+        lib.oracle_mlp_forward.argtypes = [vp, i64, i64, i64, vp, vp, vp, vp, vp, vp, vp, i64, vp, vp, c_int]
         lib.oracle_default_threads.restype = c_int
         lib.oracle_default_threads.argtypes = []
         self.lib = lib
@@ -144,6 +147,34 @@ class Oracle:
             out["h"] = h
         return out
 
+    def mlp_forward(self, x_bits, q1, s1, q3, s3, q2, s2, tokens=None, threads: int = 0,
+                    want_hidden: bool = False):
+        """The dense ExpertsInt8 MLP in fp64 on the listed tokens (all if None).
+
+        x [T][d] bf16 bits; q1, q3 [F][d] int8 with s1, s3 [F] fp32; q2 [d][F] int8 with s2 [d] fp32.
+        Returns a dict with y fp64 [n][d] and, if asked, h fp64 [n][F].
+        """
+        x = _c(x_bits, np.uint16)
+        q1, q3, q2 = (_c(a, np.int8) for a in (q1, q3, q2))
+        s1, s3, s2 = (_c(a, np.float32) for a in (s1, s3, s2))
+        T, d = x.shape
+        F = q1.shape[0]
+        assert q1.shape == (F, d) and q3.shape == (F, d) and q2.shape == (d, F)
+        assert s1.shape == (F,) and s3.shape == (F,) and s2.shape == (d,)
+        tok = None if tokens is None else np.ascontiguousarray(tokens, dtype=np.int64)
+        n = T if tok is None else tok.size
+        y = np.empty((n, d), dtype=np.float64)
+        h = np.empty((n, F), dtype=np.float64) if want_hidden else None
+        rc = self.lib.oracle_mlp_forward(x.ctypes.data, T, d, F, q1.ctypes.data, s1.ctypes.data, q3.ctypes.data,
+                                         s3.ctypes.data, q2.ctypes.data, s2.ctypes.data, _ptr(tok), n,
+                                         y.ctypes.data, _ptr(h), threads)
+        if rc != 0:
+            raise ValueError("oracle_mlp_forward rejected its arguments")
+        out = {"y": y}
+        if want_hidden:
+            out["h"] = h
+        return out
+
 
 _default: Optional[Oracle] = None
 
@@ -173,3 +204,7 @@ def moe_forward(*args, **kwargs):
 
 def moe_forward_bf16w(*args, **kwargs):
     return get().moe_forward_bf16w(*args, **kwargs)
+
+
+def mlp_forward(*args, **kwargs):
+    return get().mlp_forward(*args, **kwargs)

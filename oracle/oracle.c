@@ -28,6 +28,9 @@
  *     q * scale formed exactly in fp64 (Jamba-1.5 paper, §3.1: weights are
  *     dequantized back before the computation).  No intermediate rounding:
  *     the result is fp64.
+ *   - oracle_mlp_forward: the dense MLP of the layers without MoE, whose weights
+ *     ExpertsInt8 quantizes too (Jamba-1.5 paper, §3.1): the same SwiGLU block
+ *     as one expert, every token with weight 1.
  *
  * Parity pins: every function here is checked by the `-m "not gpu"` tests
  * against exact rational arithmetic, closed forms, invariants and brute-force
@@ -388,6 +391,50 @@ int oracle_moe_forward_bf16w(const uint16_t* x, int64_t T, int64_t d, int64_t F,
     }
     fwdb_ctx c = {x, d, F, E, K, wr, bias, w1, w3, w2, tokens, y, ids, wts, h_out};
     parallel_for(n_tokens, threads, forward_bf16w_range, &c);
+    return 0;
+}
+
+/* ------------------------------------------------------------- dense MLP */
+
+/* The MLP of a layer without MoE, with ExpertsInt8 weights (Jamba-1.5 paper, §3.1 "ExpertsInt8":
+ * the MLP weights are quantized like the experts'; "Model Architecture": MoE replaces the single
+ * MLP only every e = 2 layers).  The MLP is the same SwiGLU block as one expert,
+ *   y_t = W2 (SiLU(W1 x_t) * (W3 x_t)),  w = q * scale formed exactly in fp64,
+ * taken by every token with weight 1: no router, no softmax, no sum over experts. */
+static void mlp_range(void* p, int64_t b, int64_t e) {
+    fwd_ctx* c = (fwd_ctx*)p;
+    const int64_t d = c->d, F = c->F;
+    double* xd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    for (int64_t n = b; n < e; ++n) {
+        const int64_t t = c->tokens ? c->tokens[n] : n;
+        const uint16_t* xt = c->x + t * d;
+        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);
+        expert_ffn(c, 0, xd, h, c->y + n * d);
+        if (c->h_out) memcpy(c->h_out + n * F, h, sizeof(double) * (size_t)F);
+    }
+    free(xd);
+    free(h);
+}
+
+/* The dense MLP on a subset of tokens.
+ *   x: bf16 bits [T][d]; q1, q3: int8 [F][d] with s1, s3 fp32 [F]; q2: int8 [d][F] with s2 fp32 [d];
+ *   tokens: int64 [n_tokens] indices into x, or NULL for tokens 0..n_tokens-1;
+ *   y: fp64 [n_tokens][d] (output); h_out: fp64 [n_tokens][F] (optional, the SwiGLU hidden).
+ * Returns 0, or -1 on bad arguments. */
+int oracle_mlp_forward(const uint16_t* x, int64_t T, int64_t d, int64_t F, const int8_t* q1, const float* s1,
+                       const int8_t* q3, const float* s3, const int8_t* q2, const float* s2, const int64_t* tokens,
+                       int64_t n_tokens, double* y, double* h_out, int threads) {
+    if (!x || !q1 || !s1 || !q3 || !s3 || !q2 || !s2 || !y) return -1;
+    if (T < 0 || d <= 0 || F <= 0 || n_tokens < 0) return -1;
+    if (tokens) {
+        for (int64_t n = 0; n < n_tokens; ++n)
+            if (tokens[n] < 0 || tokens[n] >= T) return -1;
+    } else if (n_tokens > T) {
+        return -1;
+    }
+    fwd_ctx c = {x, d, F, 1, 1, NULL, NULL, q1, q3, q2, s1, s3, s2, tokens, y, NULL, NULL, h_out};
+    parallel_for(n_tokens, threads, mlp_range, &c);
     return 0;
 }
 

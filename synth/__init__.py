@@ -26,7 +26,11 @@ STREAM_ROUTER = 2
 STREAM_W1 = 3
 STREAM_W3 = 4
 STREAM_W2 = 5
+STREAM_MLP_W1 = 6
+STREAM_MLP_W3 = 7
+STREAM_MLP_W2 = 8
 _WEIGHT_STREAM = {"w1": STREAM_W1, "w3": STREAM_W3, "w2": STREAM_W2}
+_MLP_WEIGHT_STREAM = {"w1": STREAM_MLP_W1, "w3": STREAM_MLP_W3, "w2": STREAM_MLP_W2}
 
 _lib = None
 
@@ -104,6 +108,7 @@ class Workload:
     bias: Dict[int, float] = field(default_factory=dict)  # router logit bias per expert
     seed: int = 0
     note: str = ""
+    layer: str = "moe"  # "moe": the routed expert layer; "mlp": the dense MLP (E = K = 1, no router)
 
 
 WORKLOADS: Dict[str, Workload] = {
@@ -123,6 +128,27 @@ WORKLOADS: Dict[str, Workload] = {
                  bias={3: 2.0, 11: 2.0}, note="skewed routing stress (+2.0 logit bias on experts 3 and 11)"),
     ]
 }
+
+
+# The dense MLP of the layers without MoE (Jamba-1.5 paper, "Model Architecture": MoE replaces the
+# MLP every e = 2 layers; §3.1: ExpertsInt8 quantizes the MLP weights too), with the expert's shape.
+MLP_WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in [
+        Workload("mlp_tiny", T=64, d=256, F=512, E=1, K=1, w_std=0.02, layer="mlp",
+                 note="tiny dense MLP, oracle-checkable in full"),
+        Workload("mlp_v01_decode", T=32, d=4096, F=14336, E=1, K=1, w_std=0.02, layer="mlp",
+                 note="Jamba-v0.1-shaped dense MLP, decode step (int8 weights 176 MB, HBM-bound)"),
+        Workload("mlp_v01_prefill", T=8192, d=4096, F=14336, E=1, K=1, w_std=0.02, layer="mlp",
+                 note="Jamba-v0.1-shaped dense MLP, prefill (tensor-core bound)"),
+    ]
+}
+
+ALL_WORKLOADS: Dict[str, Workload] = {**WORKLOADS, **MLP_WORKLOADS}
+
+
+def _weight_stream(wl: Workload, which: str) -> int:
+    return (_MLP_WEIGHT_STREAM if wl.layer == "mlp" else _WEIGHT_STREAM)[which]
 
 
 def weight_shape(wl: Workload, which: str):
@@ -170,7 +196,7 @@ def gen_expert(wl: Workload, which: str, e: int, seed: Optional[int] = None,
     n = rows * cols
     if out is None:
         out = np.empty((rows, cols), dtype=np.uint16)
-    normal_bf16(seed, _WEIGHT_STREAM[which], 0, e * n, n, wl.w_std, out.reshape(-1), threads)
+    normal_bf16(seed, _weight_stream(wl, which), 0, e * n, n, wl.w_std, out.reshape(-1), threads)
     return out
 
 
@@ -179,5 +205,5 @@ def gen_experts(wl: Workload, which: str, seed: Optional[int] = None) -> np.ndar
     rows, cols = weight_shape(wl, which)
     out = np.empty((wl.E, rows, cols), dtype=np.uint16)
     seed = wl.seed if seed is None else seed
-    normal_bf16(seed, _WEIGHT_STREAM[which], 0, 0, out.size, wl.w_std, out.reshape(-1))
+    normal_bf16(seed, _weight_stream(wl, which), 0, 0, out.size, wl.w_std, out.reshape(-1))
     return out

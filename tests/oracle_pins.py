@@ -318,4 +318,54 @@ def pin_bf16w_identical_experts_is_dense_mlp(orc):
     assert np.allclose(out["y"], y_ref, rtol=1e-12, atol=1e-15)
 
 
+# ------------------------------------------------------------- dense MLP
+
+
+def tiny_mlp(rng, T=6, d=32, F=40, wstd=0.05):
+    L = tiny_layer(rng, T=T, d=d, F=F, E=1, wstd=wstd)
+    return {k: (np.ascontiguousarray(v[0]) if k not in ("x", "wr") else v) for k, v in L.items()}
+
+
+def mlp(orc, L, **kw):
+    return orc.mlp_forward(L["x"], L["q1"], L["s1"], L["q3"], L["s3"], L["q2"], L["s2"], **kw)
+
+
+def pin_mlp_matches_torch_swiglu(orc):
+    L = tiny_mlp(np.random.default_rng(31), T=7, d=40, F=56)
+    out = mlp(orc, L, want_hidden=True)
+    y_ref, h_ref = swiglu_torch(synth.bf16_bits_to_f32(L["x"]), dequant(L["q1"], L["s1"]),
+                                dequant(L["q3"], L["s3"]), dequant(L["q2"], L["s2"]))
+    assert np.allclose(out["h"], h_ref, rtol=1e-12, atol=1e-15)
+    assert np.allclose(out["y"], y_ref, rtol=1e-12, atol=1e-15)
+
+
+def pin_mlp_zero_gate_or_up_and_exact_scaling(orc):
+    L = tiny_mlp(np.random.default_rng(32))
+    y = mlp(orc, L)["y"]
+    for key in ("q1", "q3"):
+        M = dict(L)
+        M[key] = np.zeros_like(L[key])
+        assert not np.any(mlp(orc, M)["y"]), key
+    for key in ("s2", "s3"):
+        M = dict(L)
+        M[key] = L[key] * np.float32(2.0)
+        assert np.array_equal(mlp(orc, M)["y"], 2.0 * y), key
+
+
+def pin_mlp_one_hot_and_token_subset(orc):
+    L = tiny_mlp(np.random.default_rng(33), T=9, d=16, F=24)
+    full = mlp(orc, L)["y"]
+    sub = [8, 2, 5]
+    assert np.array_equal(mlp(orc, L, tokens=sub)["y"], full[sub])
+    i = 5
+    x = np.zeros((1, 16), np.float32)
+    x[0, i] = 1.0
+    M = dict(L)
+    M["x"] = bf16_bits(x)
+    out = mlp(orc, M, want_hidden=True)
+    a1 = torch.as_tensor(L["q1"][:, i].astype(np.float64) * L["s1"].astype(np.float64))
+    a3 = L["q3"][:, i].astype(np.float64) * L["s3"].astype(np.float64)
+    assert np.allclose(out["h"][0], torch.nn.functional.silu(a1).numpy() * a3, rtol=1e-14, atol=0)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

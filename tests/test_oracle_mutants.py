@@ -28,6 +28,9 @@ MUTANTS = {
     "bf16w_down_transposed": ("acc += (double)bf16_value(r2[j]) * h[j];",
                               "acc += (double)bf16_value(w2[j * d + i]) * h[j];"),
     "bf16w_up_uses_gate": ("a3 += (double)bf16_value(r3[i]) * xd[i];", "a3 += (double)bf16_value(r1[i]) * xd[i];"),
+    "mlp_output_row_by_token": ("expert_ffn(c, 0, xd, h, c->y + n * d);", "expert_ffn(c, 0, xd, h, c->y + t * d);"),
+    "mlp_first_token_only": ("xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn",
+                             "xt = c->x;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn"),
     "router_ignores_last_input": ("for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i])",
                                   "for (int64_t i = 0; i + 1 < d; ++i) acc += (double)bf16_value(x[i])"),
 }

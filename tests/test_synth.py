@@ -68,3 +68,13 @@ def test_workloads_shapes():
     assert np.array_equal(np.delete(x2, 5, 0), np.delete(x, 5, 0))
     assert not np.array_equal(x2[5], x[5])
     assert synth.gen_bias(synth.WORKLOADS["skewed"])[[3, 11]].tolist() == [2.0, 2.0]
+
+
+def test_mlp_workloads_draw_their_own_weights():
+    wl = synth.MLP_WORKLOADS["mlp_tiny"]
+    assert wl.E == 1 and wl.K == 1 and wl.layer == "mlp"
+    w1 = synth.gen_experts(wl, "w1")
+    assert w1.shape == (1, 512, 256)
+    # same shape as the tiny MoE layer's expert 0, but another stream
+    assert not np.array_equal(w1[0], synth.gen_expert(synth.WORKLOADS["tiny"], "w1", 0))
+    assert set(synth.ALL_WORKLOADS) == set(synth.WORKLOADS) | set(synth.MLP_WORKLOADS)
