@@ -28,6 +28,7 @@ import numpy as np  # noqa: E402
 import synth  # noqa: E402
 
 METRIC = "MoE-layer tokens/sec (int8 experts) at 1 B200; % of HBM / BF16 roofline"
+METRIC_MLP = "dense-MLP tokens/sec (ExpertsInt8 weights) at 1 B200; % of HBM / BF16 roofline"
 UNIT = "tokens/s"
 DEFAULT_WORKLOAD = "v01_decode"
 
@@ -37,7 +38,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.ALL_WORKLOADS),
+                    help="MoE layer workloads, or mlp_* for the dense ExpertsInt8 MLP")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--weights", default="int8", choices=["int8", "bf16"],
@@ -67,6 +69,11 @@ def algorithmic(kind, wl, T, touched, rows_padded, wbytes=1):
     wbytes = bytes per weight (1: int8 codes, plus 4-byte scales per row; 2: bf16, no scales)."""
     d, F, TK = wl.d, wl.F, T * wl.K
     sc = 4 if wbytes == 1 else 0
+    if wl.layer == "mlp":  # one weight matrix set, every token once (K = 1); y written in bf16 by gemv2/gemm2
+        if kind == "gemv2":
+            return "bytes", d * F * wbytes + d * sc + T * F * 2 + T * d * 2
+        if kind == "permute":
+            return "bytes", rows_padded * 4 + T * 4
     if kind == "gemv13":
         return "bytes", touched * (2 * F * d * wbytes + 2 * F * sc) + TK * d * 2 + TK * F * 2
     if kind == "gemv2":
@@ -174,7 +181,7 @@ def oracle_setup(wl, seed_x):
     """Host copies for the oracle: bf16 x, router, and the oracle's own quantization of the weights."""
     import oracle
     x = synth.gen_x(synth_replace(wl, seed=seed_x))
-    wr = synth.gen_router(wl)
+    wr = synth.gen_router(wl) if wl.layer == "moe" else None
     bias = synth.gen_bias(wl)
     qs = {}
     for which in ("w1", "w3", "w2"):
@@ -192,20 +199,31 @@ def synth_replace(wl, **kw):
     return dataclasses.replace(wl, **kw)
 
 
+def oracle_forward(wl, setup, tokens, threads):
+    """The oracle's layer (the MoE layer, or the dense MLP for mlp_* workloads) on the listed tokens."""
+    import oracle
+    x, wr, bias, qs = setup
+    if wl.layer == "mlp":
+        q1, s1 = qs["w1"]
+        q3, s3 = qs["w3"]
+        q2, s2 = qs["w2"]
+        return oracle.mlp_forward(x, q1[0], s1[0], q3[0], s3[0], q2[0], s2[0], tokens=tokens, threads=threads)
+    return oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=tokens, threads=threads)
+
+
 def oracle_rate(wl, setup, budget_s, max_tokens=None):
     """Tokens/s of the oracle forward on a bounded sample (tokens spread over the batch)."""
     import oracle
-    x, wr, bias, qs = setup
     threads = oracle.default_threads()
     t0 = time.perf_counter()
-    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=[0], threads=1)
+    oracle_forward(wl, setup, [0], 1)
     per_token_1t = time.perf_counter() - t0
     n = max(1, min(wl.T, int(budget_s * threads / max(per_token_1t, 1e-9))))
     if max_tokens:
         n = min(n, max_tokens)
     toks = np.linspace(0, wl.T - 1, n).round().astype(np.int64)
     t0 = time.perf_counter()
-    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+    oracle_forward(wl, setup, toks, threads)
     dt = time.perf_counter() - t0
     used = min(threads, n)
     return n / dt, used, n, dt
@@ -215,28 +233,27 @@ def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.ALL_WORKLOADS[args.workload]
     setup = oracle_setup(wl, wl.seed)
     import oracle
     threads = oracle.default_threads()
     # calibrate one token on one thread, then size every step to fit a few minutes in total
-    x, wr, bias, qs = setup
     t0 = time.perf_counter()
-    oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=[0], threads=1)
+    oracle_forward(wl, setup, [0], 1)
     per_tok = time.perf_counter() - t0
     step_budget = min(args.cpu_budget_s, 150.0 / max(1, args.steps + args.warmup))
     n = int(max(1, min(wl.T, step_budget * threads / per_tok)))
     toks = np.linspace(0, wl.T - 1, n).round().astype(np.int64)
     for _ in range(args.warmup):
-        oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+        oracle_forward(wl, setup, toks, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.moe_forward(x, wr, bias, *qs["w1"], *qs["w3"], *qs["w2"], tokens=toks, threads=threads)
+        oracle_forward(wl, setup, toks, threads)
     dt = time.perf_counter() - t0
     value = n * args.steps / dt
     sample = f"{n} of {wl.T} tokens per step (evenly spaced), full fp64 layer per token"
     out = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC if wl.layer == "moe" else METRIC_MLP, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": workload_config(wl, "oracle"),
@@ -249,7 +266,8 @@ def run_reference(args):
 
 
 def workload_config(wl, path):
-    return {"workload": wl.name, "T": wl.T, "d": wl.d, "ffn": wl.F, "experts": wl.E, "top_k": wl.K,
+    return {"workload": wl.name, "layer": wl.layer, "T": wl.T, "d": wl.d, "ffn": wl.F, "experts": wl.E,
+            "top_k": wl.K,
             "weights": "int8 codes + fp32 per-output-channel scales", "activations": "bf16",
             "path": path, "l2": l2_note(wl)}
 
@@ -296,7 +314,10 @@ def run_ours(args):
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.ALL_WORKLOADS[args.workload]
+    mlp = wl.layer == "mlp"
+    if mlp and args.weights != "int8":
+        raise SystemExit("the dense MLP workloads run with ExpertsInt8 weights only")
     T, d, F, E = wl.T, wl.d, wl.F, wl.E
     path = {"auto": jm.PATH_AUTO, "gemv": jm.PATH_GEMV, "gemm": jm.PATH_GEMM}[args.path]
     peaks = load_peaks()
@@ -306,7 +327,7 @@ def run_ours(args):
     x_bits = synth.gen_x(synth_replace(wl, seed=seed_x))
     to_dev = lambda b: torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).to(dev).view(torch.bfloat16)  # noqa
     x = to_dev(x_bits)
-    wr = torch.from_numpy(synth.gen_router(wl)).to(dev)
+    wr = None if mlp else torch.from_numpy(synth.gen_router(wl)).to(dev)
     bias_np = synth.gen_bias(wl)
     bias = None if bias_np is None else torch.from_numpy(bias_np).to(dev)
     int8w = args.weights == "int8"
@@ -332,14 +353,18 @@ def run_ours(args):
     q_ms = jm.jamba_moe_timing_collect().get("quantize", (0.0, 0))[0]
     jm.jamba_moe_timing_start(0)
     q_bytes = algorithmic("quantize", wl, T, 0, 0)[1]
-    ws = torch.empty(jm.jamba_moe_workspace_size(T, d, F), dtype=torch.uint8, device=dev)
+    ws_bytes = jm.jamba_mlp_workspace_size(T, d, F) if mlp else jm.jamba_moe_workspace_size(T, d, F)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     ids = torch.empty((T, 2), dtype=torch.int32, device=dev)
     tw = torch.empty((T, 2), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def forward(xin):
-        if int8w:
+        if mlp:
+            jm.jamba_mlp_forward(xin, Q["w1"][0], S["w1"][0], Q["w3"][0], S["w3"][0], Q["w2"][0], S["w2"][0], y=y,
+                                 workspace=ws, path=path)
+        elif int8w:
             jm.jamba_moe_forward(xin, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
                                  topk_ids=ids, topk_w=tw, workspace=ws, path=path)
         else:
@@ -357,7 +382,7 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
     status = jm.jamba_moe_read_device_status(ws)
-    ids_np = ids.cpu().numpy()
+    ids_np = np.zeros((T, 1), np.int32) if mlp else ids.cpu().numpy()
     touched = int(np.unique(ids_np).size)
     counts = np.bincount(ids_np.reshape(-1), minlength=E)
     rows_padded = int(sum((c + 127) // 128 * 128 for c in counts))
@@ -430,7 +455,8 @@ def run_ours(args):
 
     if rank == 0:
         out = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "metric": METRIC_MLP if mlp else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",

@@ -136,6 +136,42 @@ int jamba_moe_forward_bf16w(const uint16_t* x, const float* router_W, const floa
                             void* workspace, size_t workspace_bytes, void* stream, int path);
 
 /*
+ * jamba_mlp_workspace_size — bytes of device scratch jamba_mlp_forward needs for these sizes.
+ * Returns 0 for unsupported sizes.  Host only; touches no device.
+ */
+size_t jamba_mlp_workspace_size(int64_t T, int64_t d, int64_t ffn);
+
+/*
+ * jamba_mlp_forward — the dense MLP of the layers without MoE, on ExpertsInt8 weights (Jamba-1.5
+ * paper, §3.1: the MLP weights are quantized and dequantized like the experts'; "Model
+ * Architecture": MoE takes the place of the MLP only every e = 2 layers):
+ *
+ *     y_t = bf16( S2 * (Q2 . h_t) ),  h_t = bf16( SiLU(S1 * (Q1 . x_t)) * (S3 * (Q3 . x_t)) )
+ *
+ *   x:       bf16 [T][d]                        activations
+ *   Q1, Q3:  int8 [ffn][d] with S1, S3 fp32 [ffn]  (gate, up; from jamba_moe_quantize)
+ *   Q2:      int8 [d][ffn] with S2 fp32 [d]        (down)
+ *   y:       bf16 [T][d]                        output (written)
+ *   workspace: device scratch of at least jamba_mlp_workspace_size(...) bytes, 256-byte aligned,
+ *            owned by the caller, contents on entry irrelevant; not shared by overlapping calls.
+ *
+ * It runs the kernels of jamba_moe_forward as a layer of one expert that every token takes with
+ * weight 1 (no router, no combine: the down-projection writes y in bf16 directly).  Numerics as
+ * in jamba_moe_forward: exact int8 -> bf16, fp32 accumulation, scales on the accumulators, h in
+ * bf16; deterministic.  Sizes: 1 <= T <= 1<<20, d and ffn multiples of 128 in [128, 32768];
+ * x, y, Q1, Q3, Q2 16-byte aligned, scales 4-byte aligned.  Errors as in jamba_moe_forward.
+ */
+int jamba_mlp_forward(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                      const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/* jamba_mlp_forward_path — jamba_mlp_forward with the path chosen explicitly (JMOE_PATH_*; AUTO
+ * takes the weight-streaming path for T <= 64 tokens, the tensor-core GEMMs above). */
+int jamba_mlp_forward_path(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                           const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y,
+                           void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/*
  * jamba_moe_read_device_status — synchronises `stream`, then returns the status word the
  * kernels of the last forward call on `workspace` left there: JMOE_OK, JMOE_DEV_TIMEOUT (a
  * pipeline wait ran out of its bounded number of polls; the kernel released its resources and

@@ -48,6 +48,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_workspace_size.argtypes = [i64, i64, i64, c_int, c_int]
     fwd_args = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, sz, vp]
     lib.jamba_moe_forward.restype = c_int
+    lib.jamba_mlp_workspace_size.restype = sz
+    lib.jamba_mlp_workspace_size.argtypes = [i64, i64, i64]
+    mlp_args = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
+    lib.jamba_mlp_forward.restype = c_int
+    lib.jamba_mlp_forward.argtypes = mlp_args
+    lib.jamba_mlp_forward_path.restype = c_int
+    lib.jamba_mlp_forward_path.argtypes = mlp_args + [c_int]
     lib.jamba_moe_forward.argtypes = fwd_args
     lib.jamba_moe_forward_path.restype = c_int
     lib.jamba_moe_forward_path.argtypes = fwd_args + [c_int]
@@ -180,6 +187,46 @@ def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Opti
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward")
     return y, topk_ids, topk_w
+
+
+def jamba_mlp_workspace_size(T: int, d: int, ffn: int) -> int:
+    return int(load_library().jamba_mlp_workspace_size(T, d, ffn))
+
+
+def jamba_mlp_forward(x: torch.Tensor, Q1: torch.Tensor, S1: torch.Tensor, Q3: torch.Tensor, S3: torch.Tensor,
+                      Q2: torch.Tensor, S2: torch.Tensor, y: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                      path: int = PATH_AUTO) -> torch.Tensor:
+    """The dense ExpertsInt8 MLP on x [T][d] (bf16): Q1, Q3 int8 [ffn][d] with S1, S3 fp32 [ffn];
+    Q2 int8 [d][ffn] with S2 fp32 [d] (from jamba_moe_quantize).  Returns y bf16 [T][d].
+    ``workspace`` (uint8, >= jamba_mlp_workspace_size bytes) is allocated when not given."""
+    lib = load_library()
+    _check(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be [T][d]")
+    T, d = x.shape
+    ffn = Q1.shape[0]
+    _check(Q1, "Q1", torch.int8, (ffn, d))
+    _check(Q3, "Q3", torch.int8, (ffn, d))
+    _check(Q2, "Q2", torch.int8, (d, ffn))
+    _check(S1, "S1", torch.float32, (ffn,))
+    _check(S3, "S3", torch.float32, (ffn,))
+    _check(S2, "S2", torch.float32, (d,))
+    if y is None:
+        y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device)
+    _check(y, "y", torch.bfloat16, (T, d))
+    need = jamba_mlp_workspace_size(T, d, ffn)
+    if need == 0:
+        raise JmoeError(2, "jamba_mlp_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    st = lib.jamba_mlp_forward_path(x.data_ptr(), Q1.data_ptr(), S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(),
+                                    Q2.data_ptr(), S2.data_ptr(), T, d, ffn, y.data_ptr(), workspace.data_ptr(),
+                                    workspace.numel(), _stream_ptr(stream), int(path))
+    if st != 0:
+        raise JmoeError(st, "jamba_mlp_forward")
+    return y
 
 
 def jamba_moe_forward_bf16w(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor],

@@ -33,9 +33,17 @@ cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_
 cudaError_t launch_combine(const float* slots, int64_t T, int64_t d, uint16_t* y, cudaStream_t st, int num_sms);
 cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
-                          int64_t d, int64_t F, cudaStream_t st);
+                          int64_t d, int64_t F, cudaStream_t st, int n_exp);
 cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2, const float* S2,
-                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st);
+                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st,
+                         int n_exp, uint16_t* y);
+cudaError_t launch_dense_setup(int64_t T, WsHeader* hdr, int32_t* perm, float* wts, cudaStream_t st, int num_sms);
+cudaError_t launch_gemv13_dense(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
+                                const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T,
+                                int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemv2_dense(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
+                               const float* S2, const float* wts, uint16_t* y, int64_t T, int64_t d, int64_t F,
+                               cudaStream_t st);
 
 namespace {
 
@@ -220,13 +228,13 @@ int forward_impl(const uint16_t* x, const float* router_W, const float* router_b
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
         {
             TimedLaunch t(JMOE_KERNEL_GEMM13, st);
-            e = w8 ? launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st)
+            e = w8 ? launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st, kExperts)
                    : launch_gemm13_bf16w(hdr, perm, x_perm, B1, B3, h, L.rows_cap, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
         {
             TimedLaunch t(JMOE_KERNEL_GEMM2, st);
-            e = w8 ? launch_gemm2(hdr, perm, h, Q2, S2, wts, slots, L.rows_cap, d, ffn, st)
+            e = w8 ? launch_gemm2(hdr, perm, h, Q2, S2, wts, slots, L.rows_cap, d, ffn, st, kExperts, nullptr)
                    : launch_gemm2_bf16w(hdr, perm, h, B2, wts, slots, L.rows_cap, d, ffn, st);
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
@@ -240,7 +248,107 @@ int forward_impl(const uint16_t* x, const float* router_W, const float* router_b
 
 }  // namespace
 
+namespace {
+
+// ---------------------------------------------------------------- dense MLP
+// The MLP runs as a one-expert layer: a table kernel in place of router + permute, the same
+// expert kernels, and a down-projection that writes y in bf16 (no slots, no combine).
+constexpr int64_t kMlpGemvMaxTokens = 64;
+
+Layout make_layout_mlp(int64_t T, int64_t d, int64_t F) {
+    Layout L{};
+    L.rows_cap = (T + kRowPad - 1) / kRowPad * kRowPad;
+    size_t off = 0;
+    L.hdr = off;
+    off = align256(off + kHeaderBytes);
+    L.wts = off;
+    off = align256(off + sizeof(float) * T * kTopK);
+    L.perm = off;
+    off = align256(off + sizeof(int32_t) * L.rows_cap);
+    L.x_perm = off;
+    off = align256(off + sizeof(uint16_t) * L.rows_cap * d);
+    L.h = off;
+    off = align256(off + sizeof(uint16_t) * L.rows_cap * F);
+    L.ids = L.inv = L.slots = off;  // unused
+    L.total = off;
+    return L;
+}
+
+int mlp_impl(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+             const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y, void* workspace,
+             size_t workspace_bytes, void* stream, int path) {
+    if (!x || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
+    if (!shape_ok(T, d, ffn, kExperts, kTopK)) return JMOE_ERR_SHAPE;
+    if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    const void* ptrs16[] = {x, Q1, Q3, Q2, y};
+    for (const void* p : ptrs16)
+        if (!aligned16(p)) return JMOE_ERR_ALIGN;
+    const void* ptrs4[] = {S1, S3, S2};
+    for (const void* p : ptrs4)
+        if (reinterpret_cast<uintptr_t>(p) & 3) return JMOE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return JMOE_ERR_WORKSPACE;
+    const Layout L = make_layout_mlp(T, d, ffn);
+    if (workspace_bytes < L.total) return JMOE_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+    float* wts = reinterpret_cast<float*>(ws + L.wts);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = num_sms_current();
+    if (path == JMOE_PATH_AUTO) path = (T <= kMlpGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
+
+    cudaError_t e;
+    {
+        TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
+        e = launch_dense_setup(T, hdr, perm, wts, st, sms);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (path == JMOE_PATH_GEMV) {
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV13, st);
+            e = launch_gemv13_dense(hdr, perm, x, Q1, S1, Q3, S3, h, T, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        TimedLaunch t(JMOE_KERNEL_GEMV2, st);
+        return to_status(launch_gemv2_dense(hdr, perm, h, Q2, S2, wts, y, T, d, ffn, st));
+    }
+    {
+        TimedLaunch t(JMOE_KERNEL_GATHER, st);
+        e = launch_gather(x, perm, hdr, d, L.rows_cap, x_perm, st, sms, true);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_GEMM13, st);
+        e = launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st, 1);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    TimedLaunch t(JMOE_KERNEL_GEMM2, st);
+    return to_status(launch_gemm2(hdr, perm, h, Q2, S2, wts, nullptr, L.rows_cap, d, ffn, st, 1, y));
+}
+
+}  // namespace
+
 extern "C" {
+
+size_t jamba_mlp_workspace_size(int64_t T, int64_t d, int64_t ffn) {
+    if (!shape_ok(T, d, ffn, kExperts, kTopK)) return 0;
+    return make_layout_mlp(T, d, ffn).total;
+}
+
+int jamba_mlp_forward_path(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                           const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y,
+                           void* workspace, size_t workspace_bytes, void* stream, int path) {
+    return mlp_impl(x, Q1, S1, Q3, S3, Q2, S2, T, d, ffn, y, workspace, workspace_bytes, stream, path);
+}
+
+int jamba_mlp_forward(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                      const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    return mlp_impl(x, Q1, S1, Q3, S3, Q2, S2, T, d, ffn, y, workspace, workspace_bytes, stream, JMOE_PATH_AUTO);
+}
 
 int jamba_moe_forward_path(const uint16_t* x, const float* router_W, const float* router_bias, const int8_t* Q1,
                            const float* S1, const int8_t* Q3, const float* S3, const int8_t* Q2, const float* S2,

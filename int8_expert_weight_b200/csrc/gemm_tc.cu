@@ -48,6 +48,7 @@ struct GemmArgs {
     int band;             // M tiles per raster band
     uint32_t max_polls;   // bound of every mbarrier wait
     int skip_copy;        // test hook: CTA 0 skips the copies of its second K step (a wait then runs out)
+    uint16_t* y_out;      // gemm2 of the dense MLP: y [T][N] in bf16, written instead of out_slot
 };
 
 // Shared-memory ring: per stage the activation tile, the bf16 weight tile the MMA reads and, for
@@ -339,22 +340,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 const int32_t a = p.perm[gr];
                 const float wt = a >= 0 ? p.wts[a] : 0.0f;
                 const float* s2 = p.sa + (int64_t)t.e * p.N + i0;
-                float* orow = p.slot_out + (int64_t)(a >= 0 ? a : 0) * p.N + i0;
+                if (p.y_out) {
+                    // dense MLP: one assignment per token, its output rounded to bf16 here
+                    uint16_t* yrow = p.y_out + (int64_t)(a >= 0 ? a / kTopK : 0) * p.N + i0;
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v[32];
-                    tc::tmem_ld32(tbase + c, v);
-                    tc::tmem_wait_ld();
-                    if (a >= 0) {
-                        float4* dst = reinterpret_cast<float4*>(orow + c);
+                    for (int c = 0; c < BN; c += 32) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tbase + c, v);
+                        tc::tmem_wait_ld();
+                        if (a >= 0) {
+                            uint32_t packed[16];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            float4 o;
-                            o.x = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
-                            o.y = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
-                            o.z = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
-                            o.w = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
-                            dst[k] = o;
+                            for (int i = 0; i < 32; i += 2) {
+                                const float o0 = wt * ((kW8 ? __ldg(s2 + c + i) : 1.0f) * __uint_as_float(v[i]));
+                                const float o1 =
+                                    wt * ((kW8 ? __ldg(s2 + c + i + 1) : 1.0f) * __uint_as_float(v[i + 1]));
+                                packed[i / 2] =
+                                    (uint32_t)f32_to_bf16_bits(o0) | ((uint32_t)f32_to_bf16_bits(o1) << 16);
+                            }
+                            uint4* dst = reinterpret_cast<uint4*>(yrow + c);
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2],
+                                                    packed[4 * k + 3]);
+                        }
+                    }
+                } else {
+                    float* orow = p.slot_out + (int64_t)(a >= 0 ? a : 0) * p.N + i0;
+#pragma unroll 1
+                    for (int c = 0; c < BN; c += 32) {
+                        uint32_t v[32];
+                        tc::tmem_ld32(tbase + c, v);
+                        tc::tmem_wait_ld();
+                        if (a >= 0) {
+                            float4* dst = reinterpret_cast<float4*>(orow + c);
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                float4 o;
+                                o.x = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
+                                o.y = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
+                                o.z = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
+                                o.w = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
+                                dst[k] = o;
+                            }
                         }
                     }
                 }
@@ -454,16 +482,17 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
 
 }  // namespace
 
-// h = SwiGLU(x_perm . Q1^T, x_perm . Q3^T) per expert segment; rows_cap = permuted-row capacity.
+// h = SwiGLU(x_perm . Q1^T, x_perm . Q3^T) per expert segment; rows_cap = permuted-row capacity;
+// n_exp = experts held by Q1/Q3 (16, or 1 for the dense MLP).
 cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
-                          int64_t d, int64_t F, cudaStream_t st) {
+                          int64_t d, int64_t F, cudaStream_t st, int n_exp) {
     CUtensorMap ta, tb0, tb1;
     if (!make_map(&ta, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kBM, kBK,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tb0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, kBK,
+        !make_map(&tb0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * F, d, 128, kBK,
                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, kBK,
+        !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * F, d, 128, kBK,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,          perm,          S1,          S3,
@@ -473,19 +502,21 @@ cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_
     return launch_gemm_t<true, 256, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
-// out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment.
+// out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment, or, given y (the dense MLP, one
+// assignment per token), y[a / K] = bf16(p_a * S2 . (h_perm . Q2^T)).
 cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2, const float* S2,
-                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st) {
+                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st,
+                         int n_exp, uint16_t* y) {
     const int BN = (d % 256 == 0) ? 256 : 128;
     CUtensorMap ta, tb0;
     if (!make_map(&ta, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * d, F, BN, kBK,
+        !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * d, F, BN, kBK,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,         perm,         S2,          nullptr,
                wts,         nullptr,      out_slot,    (int)F,
                (int)d,      (int)(d / BN), band_for((int)F), g_skip_copy ? kTestMaxPolls : kMaxPolls,
-               0};
+               0,           y};
     if (BN == 256) return launch_gemm_t<false, 256, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }

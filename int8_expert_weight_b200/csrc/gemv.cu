@@ -35,6 +35,7 @@ struct GemvArgs {
     float* slot_out;       // gemv2: out_slot [T*K][d]
     int64_t K;             // reduction length: d (gemv13) or F (gemv2)
     int64_t N;             // weight rows per expert: F (gemv13) or d (gemv2)
+    uint16_t* y_out;       // gemv2 of the dense MLP: y [T][d] in bf16, written instead of out_slot
 };
 
 // One k-step (16 consecutive k per lane) of weights for rows g and g+8: int8 codes fill one
@@ -239,7 +240,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32,
             } else {
                 const int32_t a = p.perm[row0 + n];
                 const float v = kW8 ? p.sa[(int64_t)e * p.N + jr] * red[o] : red[o];
-                p.slot_out[(int64_t)a * p.N + jr] = p.wts[a] * v;
+                if (p.y_out)  // one assignment per token: round its output to bf16 here
+                    p.y_out[(int64_t)(a / kTopK) * p.N + jr] = f32_to_bf16_bits(p.wts[a] * v);
+                else
+                    p.slot_out[(int64_t)a * p.N + jr] = p.wts[a] * v;
             }
         }
         __syncthreads();  // red is reused by the next pass
@@ -251,9 +255,12 @@ static int gemv_nt(int64_t T) {
     return avg <= 6 ? 1 : (avg <= 12 ? 2 : 4);
 }
 
+// Tokens per pass of the dense MLP, where all T tokens take the one weight matrix.
+static int gemv_nt_dense(int64_t T) { return T <= 8 ? 1 : (T <= 16 ? 2 : 4); }
+
 template <bool kDual, bool kW8>
-static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st) {
-    dim3 grid((unsigned)(p.N / kGemvRows), kExperts);
+static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st, int experts = kExperts) {
+    dim3 grid((unsigned)(p.N / kGemvRows), (unsigned)experts);
     if (nt == 1) return launch_pdl(gemv_kernel<1, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
     if (nt == 2) return launch_pdl(gemv_kernel<2, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
     return launch_pdl(gemv_kernel<4, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
@@ -284,6 +291,22 @@ cudaError_t launch_gemv2_bf16w(const WsHeader* hdr, const int32_t* perm, const u
                                const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F, cudaStream_t st) {
     GemvArgs p{hdr, perm, h, W2, nullptr, nullptr, nullptr, wts, nullptr, out_slot, F, d};
     return launch_gemv_t<false, false>(p, gemv_nt(T), st);
+}
+
+// The dense MLP (one weight matrix, every token with weight 1): one expert's rows of CTAs, and
+// gemv2 writes y in bf16 directly.
+cudaError_t launch_gemv13_dense(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
+                                const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T,
+                                int64_t d, int64_t F, cudaStream_t st) {
+    GemvArgs p{hdr, perm, x, Q1, Q3, S1, S3, nullptr, h, nullptr, d, F, nullptr};
+    return launch_gemv_t<true, true>(p, gemv_nt_dense(T), st, 1);
+}
+
+cudaError_t launch_gemv2_dense(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
+                               const float* S2, const float* wts, uint16_t* y, int64_t T, int64_t d, int64_t F,
+                               cudaStream_t st) {
+    GemvArgs p{hdr, perm, h, Q2, nullptr, S2, nullptr, wts, nullptr, nullptr, F, d, y};
+    return launch_gemv_t<false, true>(p, gemv_nt_dense(T), st, 1);
 }
 
 }  // namespace jmoe

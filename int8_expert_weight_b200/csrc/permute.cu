@@ -128,6 +128,41 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     }
 }
 
+// The routing table of the dense MLP, which every token takes with weight 1: the MLP is run as a
+// one-expert layer whose expert 0 holds all T tokens in token order.  Token t is assignment t*K
+// (the other K-1 assignment slots of a token stay unused), with weight 1; rows T.. of the segment,
+// up to the next multiple of kRowPad, are padding (-1).
+__global__ void __launch_bounds__(256) dense_setup_kernel(int64_t T, WsHeader* __restrict__ hdr,
+                                                          int32_t* __restrict__ perm, float* __restrict__ wts) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t R = (T + kRowPad - 1) / kRowPad * kRowPad;
+    if (blockIdx.x == 0 && threadIdx.x < kExperts) {
+        const int e = threadIdx.x;
+        if (e == 0) hdr->status = 0;  // first kernel of a forward call to touch the header
+        hdr->counts[e] = (e == 0) ? (int32_t)T : 0;
+        hdr->seg_start[e] = (e == 0) ? 0 : (int32_t)R;
+        hdr->tile_start[e] = (e == 0) ? 0 : (int32_t)(R / kRowPad);
+        hdr->touched[e] = (e == 0) ? 0 : -1;
+        if (e == 0) {
+            hdr->seg_start[kExperts] = (int32_t)R;
+            hdr->tile_start[kExperts] = (int32_t)(R / kRowPad);
+            hdr->n_touched = 1;
+        }
+    }
+    for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R; r += (int64_t)gridDim.x * blockDim.x) {
+        perm[r] = (r < T) ? (int32_t)(r * kTopK) : -1;
+        if (r < T) wts[r * kTopK] = 1.0f;
+    }
+}
+
+cudaError_t launch_dense_setup(int64_t T, WsHeader* hdr, int32_t* perm, float* wts, cudaStream_t st, int num_sms) {
+    const int64_t R = (T + kRowPad - 1) / kRowPad * kRowPad;
+    int64_t blocks = (R + 255) / 256;
+    if (blocks > num_sms) blocks = num_sms;
+    return launch_pdl(dense_setup_kernel, dim3((unsigned)blocks), dim3(256), 0, st, T, hdr, perm, wts);
+}
+
 cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
                            cudaStream_t st) {
     return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), 0, st, ids, T * kTopK, hdr, perm, inv);

@@ -48,6 +48,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const uint16_t* __re
     for (int64_t r = warp; r < rows; r += nwarps) {
         const uint16_t* wr = W + r * cols;
         uint32_t amax_bits = 0;  // max of |w| as an IEEE bit pattern (monotone for non-negative floats)
+#pragma unroll 4
         for (int64_t c = lane; c < chunks; c += 32) {
             const uint4 a = ld_nc_v4(wr + c * 16);
             const uint4 b = ld_nc_v4(wr + c * 16 + 8);
@@ -89,7 +90,7 @@ cudaError_t launch_quantize(const uint16_t* W, int64_t rows, int64_t cols, int8_
                             int num_sms) {
     const int threads = 256;
     int64_t blocks = (rows + 7) / 8;
-    const int64_t cap = (int64_t)num_sms * 8;
+    const int64_t cap = (int64_t)num_sms * 16;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     quantize_rows_kernel<<<(unsigned)blocks, threads, 0, st>>>(W, rows, cols, Q, S);

@@ -24,13 +24,13 @@ def declared_functions():
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names |= set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(jamba_moe_[a-z_0-9]+)\s*\(", src, re.M))
+            names |= set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(jamba_(?:moe|mlp)_[a-z_0-9]+)\s*\(", src, re.M))
     return sorted(names)
 
 
 def test_every_declared_symbol_is_exported(lib):
     names = declared_functions()
-    assert "jamba_moe_forward" in names and "jamba_moe_quantize" in names
+    assert "jamba_moe_forward" in names and "jamba_moe_quantize" in names and "jamba_mlp_forward" in names
     for n in names:
         assert hasattr(lib, n), n
 
@@ -73,6 +73,28 @@ def test_forward_argument_errors(lib):
     assert fwd(lib, x=FAKE + 8) == 7
     assert fwd(lib, ws=FAKE + 16) == 3
     assert fwd(lib, wsb=1024) == 3
+
+
+def mlp(lib, T=8, d=256, F=512, x=FAKE, ws=FAKE, wsb=1 << 40, path=0, y=FAKE, s=FAKE):
+    return lib.jamba_mlp_forward_path(x, FAKE, s, FAKE, FAKE, FAKE, FAKE, T, d, F, y, ws, wsb, None, path)
+
+
+def test_mlp_workspace_and_argument_errors(lib):
+    a = jm.jamba_mlp_workspace_size(32, 4096, 14336)
+    assert a > 128 * 14336 * 2 and a % 256 == 0
+    assert a < jm.jamba_moe_workspace_size(32, 4096, 14336)
+    assert jm.jamba_mlp_workspace_size(0, 4096, 14336) == 0
+    assert jm.jamba_mlp_workspace_size(8, 4096, 14300) == 0
+    assert mlp(lib, x=None) == 1
+    assert mlp(lib, s=None) == 1
+    assert mlp(lib, ws=None) == 1
+    assert mlp(lib, T=0) == 2
+    assert mlp(lib, d=200) == 2
+    assert mlp(lib, path=5) == 2
+    assert mlp(lib, y=FAKE + 2) == 7
+    assert mlp(lib, s=FAKE + 2) == 7
+    assert mlp(lib, ws=FAKE + 64) == 3
+    assert mlp(lib, wsb=4096) == 3
 
 
 def test_quantize_argument_errors(lib):
