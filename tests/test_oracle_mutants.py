@@ -28,7 +28,8 @@ MUTANTS = {
     "bf16w_down_transposed": ("acc += (double)bf16_value(r2[j]) * h[j];",
                               "acc += (double)bf16_value(w2[j * d + i]) * h[j];"),
     "bf16w_up_uses_gate": ("a3 += (double)bf16_value(r3[i]) * xd[i];", "a3 += (double)bf16_value(r1[i]) * xd[i];"),
-    "mlp_output_row_by_token": ("expert_ffn(c, 0, xd, h, c->y + n * d);", "expert_ffn(c, 0, xd, h, c->y + t * d);"),
+    "mlp_ignores_token_list": ("c->tokens[n] : n;\n        const uint16_t* xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn",
+                               "n : n;\n        const uint16_t* xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn"),
     "mlp_first_token_only": ("xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn",
                              "xt = c->x;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn"),
     "router_ignores_last_input": ("for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i])",
@@ -37,6 +38,7 @@ MUTANTS = {
 
 
 def _build_mutant(name, tmp_path):
+    # every mutant must keep all memory accesses in bounds: it runs inside the test process
     old, new = MUTANTS[name]
     src = open(SRC).read()
     assert src.count(old) >= 1, f"mutation site for {name} not found"
