@@ -73,7 +73,7 @@ def test_mlp_tiny_ragged(tiny, T, path):
     assert_y_close(tiny.forward(path, T), tiny.ref(T=T), f"T={T}")
 
 
-@pytest.mark.parametrize("T,d,F", [(40, 384, 640), (130, 512, 1152)])
+@pytest.mark.parametrize("T,d,F", [(40, 384, 640), (130, 512, 1152), (5, 2048, 3072), (40, 2048, 3072)])
 @pytest.mark.parametrize("path", PATHS)
 def test_mlp_other_shapes(T, d, F, path):
     L = Mlp(mlp_workload("mlp_tiny", T=T, d=d, F=F))

@@ -51,7 +51,8 @@ def test_quantize_special_rows():
     assert sg[1] == 1.0 and not qg[1].any()
 
 
-@pytest.mark.parametrize("cols", [16, 48, 256, 4096 + 16, 24576])
+@pytest.mark.parametrize("cols", [16, 48, 256, 4096, 4096 + 16, 8192, 14336, 16384, 16384 + 16, 24576, 32768,
+                                  32768 + 16, 40000])
 def test_quantize_random_rows(cols):
     rng = np.random.default_rng(cols)
     rows = max(1, 300000 // cols)
@@ -67,6 +68,18 @@ def test_quantize_all_halfway_grid():
     row = np.concatenate([[127.0], n + 0.5, -(n + 0.5), [0.0] * 1]).astype(np.float32)
     row = row[: (row.size // 16) * 16]
     assert_quant_equal(bf16_bits(row * np.float32(2.0 ** k))[None, :])
+
+
+@pytest.mark.parametrize("reps", [1, 40, 300])
+def test_quantize_halfway_rows_of_every_length_class(reps):
+    # the halfway grid repeated: rows of 240, 9600 and 72000 weights (one warp, one CTA and the
+    # two-pass kernel per row), every value an exact tie or the row's amax
+    k = -7
+    n = np.arange(120, dtype=np.float32)
+    base = np.concatenate([[127.0], n[:119] + 0.5, -(n + 0.5)]).astype(np.float32)
+    row = np.tile(base, reps)
+    rows = np.stack([row, -row, row * np.float32(2.0 ** -3)])
+    assert_quant_equal(bf16_bits(rows * np.float32(2.0 ** k)))
 
 
 def test_quantize_full_expert_matrix():
