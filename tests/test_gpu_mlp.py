@@ -87,6 +87,16 @@ def test_mlp_deterministic(tiny):
         assert np.array_equal(a, b), path
 
 
+@pytest.mark.parametrize("T", [3, 24, 64])
+def test_mlp_decode_repeatable(T):
+    """Repeated decode calls agree bit for bit, and with the oracle."""
+    L = Mlp(mlp_workload("mlp_tiny", T=T, d=2048, F=3072))
+    a = L.forward(jm.PATH_GEMV)
+    for _ in range(3):
+        assert np.array_equal(L.forward(jm.PATH_GEMV), a)
+    assert_y_close(a, L.ref())
+
+
 def test_mlp_v01_decode_all_tokens():
     L = Mlp(mlp_workload("mlp_v01_decode"))
     ref = L.ref()
