@@ -28,6 +28,9 @@
  *     q * scale formed exactly in fp64 (Jamba-1.5 paper, §3.1: weights are
  *     dequantized back before the computation).  No intermediate rounding:
  *     the result is fp64.
+ *   - oracle_quantize_rows_fp8, oracle_moe_forward_fp8: the FP8 (E4M3) layer the
+ *     Jamba-1.5 paper compares ExpertsInt8 with (§3.1), per-channel weight scales and
+ *     per-row dynamic activation scales (reading stated beside the functions).
  *   - oracle_mlp_forward: the dense MLP of the layers without MoE, whose weights
  *     ExpertsInt8 quantizes too (Jamba-1.5 paper, §3.1): the same SwiGLU block
  *     as one expert, every token with weight 1.
@@ -435,6 +438,192 @@ int oracle_mlp_forward(const uint16_t* x, int64_t T, int64_t d, int64_t F, const
     }
     fwd_ctx c = {x, d, F, 1, 1, NULL, NULL, q1, q3, q2, s1, s3, s2, tokens, y, NULL, NULL, h_out};
     parallel_for(n_tokens, threads, mlp_range, &c);
+    return 0;
+}
+
+/* ------------------------------------------------ FP8 (E4M3) comparator layer */
+
+/* The FP8 layer the Jamba-1.5 paper compares ExpertsInt8 with (§3.1: on H100 ExpertsInt8 "matches
+ * FP8 in latency"; FP8 needs hardware FP8 and, unlike ExpertsInt8, does not keep BF16 activations).
+ * The page defines no FP8 scheme; the reading taken: both GEMM operands in OCP FP8 E4M3 (1 sign,
+ * 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite 448, subnormals
+ * m * 2^-9), weights with one fp32 scale per output channel (amax / 448), activations (x, and the
+ * SwiGLU intermediate h) with one dynamic fp32 scale per row (per token, per expert slot for h);
+ * rounding to the nearest E4M3 value, ties to the even code, saturating at +-448. */
+
+/* The value of an E4M3 code (never called with the NaN codes 0x7F, 0xFF). */
+static double e4m3_value(uint8_t code) {
+    const int e = (code >> 3) & 15, m = code & 7;
+    const double v = (e == 0) ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10); /* (1 + m/8) 2^(e-7) */
+    return (code & 0x80) ? -v : v;
+}
+
+/* The E4M3 code nearest to a finite v (ties: even code), saturating at +-448; -0 keeps its sign. */
+static uint8_t e4m3_round(double v) {
+    const uint8_t sign = signbit(v) ? 0x80 : 0;
+    const double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int e2;
+    frexp(a, &e2); /* a = f * 2^e2, f in [0.5, 1) */
+    int eb = e2 - 1;   /* floor(log2 a) */
+    if (eb < -6) eb = -6; /* below the smallest normal: the subnormal spacing 2^-9 */
+    double n = nearbyint(ldexp(a, 3 - eb)); /* a / spacing, spacing = 2^(eb-3): exact scaling, ties to even */
+    if (n >= 16.0) { /* rounded up into the next binade */
+        eb += 1;
+        n = 8.0;
+    }
+    if (eb == -6 && n < 8.0) return sign | (uint8_t)n; /* subnormal */
+    return sign | (uint8_t)(((eb + 7) << 3) | ((int)n - 8));
+}
+
+/* Per-row FP8 quantization of bf16 values: scale = amax / 448 (fp32 division), code = the E4M3
+ * rounding of the exact quotient (taken in fp64, which decides every tie exactly for a bf16 value
+ * and an fp32 scale); a row of zeros gets scale 1 and code 0. */
+static void quantize_row_fp8(const uint16_t* w, int64_t cols, uint8_t* q, float* s) {
+    float amax = 0.0f;
+    for (int64_t i = 0; i < cols; ++i) {
+        float a = fabsf(bf16_value(w[i]));
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *s = 1.0f;
+        memset(q, 0, (size_t)cols);
+        return;
+    }
+    const float scale = amax / 448.0f;
+    *s = scale;
+    for (int64_t i = 0; i < cols; ++i) q[i] = e4m3_round((double)bf16_value(w[i]) / (double)scale);
+}
+
+typedef struct {
+    const uint16_t* w;
+    int64_t cols;
+    uint8_t* q;
+    float* s;
+} quant8_ctx;
+
+static void quantize_fp8_range(void* p, int64_t b, int64_t e) {
+    quant8_ctx* c = (quant8_ctx*)p;
+    for (int64_t r = b; r < e; ++r) quantize_row_fp8(c->w + r * c->cols, c->cols, c->q + r * c->cols, c->s + r);
+}
+
+/* w: bf16 bits [rows][cols]; q: E4M3 codes [rows][cols]; s: fp32 [rows]. Returns 0, or -1. */
+int oracle_quantize_rows_fp8(const uint16_t* w, int64_t rows, int64_t cols, uint8_t* q, float* s, int threads) {
+    if (!w || !q || !s || rows < 0 || cols <= 0) return -1;
+    quant8_ctx c = {w, cols, q, s};
+    parallel_for(rows, threads, quantize_fp8_range, &c);
+    return 0;
+}
+
+/* codes[i] = e4m3_round(v[i]) and values[i] = e4m3_value(codes[i]), for tests. */
+int oracle_e4m3_round(const double* v, int64_t n, uint8_t* codes, double* values) {
+    if (!v || !codes || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        codes[i] = e4m3_round(v[i]);
+        if (values) values[i] = e4m3_value(codes[i]);
+    }
+    return 0;
+}
+
+typedef struct {
+    const uint16_t* x;
+    int64_t d, F;
+    int E, K;
+    const float* wr;
+    const float* bias;
+    const uint8_t *q1, *q3, *q2;
+    const float *s1, *s3, *s2;
+    const int64_t* tokens;
+    double* y;
+    int32_t* ids;
+    double* wts;
+    double* h_out;
+} fwd8_ctx;
+
+/* One FP8 expert on one token whose activations xd are already the dequantized E4M3 values:
+ *   a1_j = sum_i (v(q1[j][i]) s1_j) xd_i, a3_j likewise, h_j = SiLU(a1_j) a3_j,
+ *   h quantized per row (scale = fp32(amax_j |h_j|) / 448 in fp32, codes of h_j / scale),
+ *   o_i = sum_j (v(q2[i][j]) s2_i) hd_j with hd the dequantized h. */
+static void expert_ffn_fp8(const fwd8_ctx* c, int e, const double* xd, double* h, uint8_t* h8, double* o) {
+    const int64_t d = c->d, F = c->F;
+    const uint8_t* q1 = c->q1 + (int64_t)e * F * d;
+    const uint8_t* q3 = c->q3 + (int64_t)e * F * d;
+    const uint8_t* q2 = c->q2 + (int64_t)e * d * F;
+    const float* s1 = c->s1 + (int64_t)e * F;
+    const float* s3 = c->s3 + (int64_t)e * F;
+    const float* s2 = c->s2 + (int64_t)e * d;
+    double amax = 0.0;
+    for (int64_t j = 0; j < F; ++j) {
+        double a1 = 0.0, a3 = 0.0;
+        const double sc1 = (double)s1[j], sc3 = (double)s3[j];
+        for (int64_t i = 0; i < d; ++i) {
+            a1 += (e4m3_value(q1[j * d + i]) * sc1) * xd[i];
+            a3 += (e4m3_value(q3[j * d + i]) * sc3) * xd[i];
+        }
+        h[j] = a1 / (1.0 + exp(-a1)) * a3;
+        if (fabs(h[j]) > amax) amax = fabs(h[j]);
+    }
+    const float hs = (amax == 0.0) ? 1.0f : (float)amax / 448.0f;
+    for (int64_t j = 0; j < F; ++j) h8[j] = (amax == 0.0) ? 0 : e4m3_round(h[j] / (double)hs);
+    for (int64_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        const double sc2 = (double)s2[i];
+        for (int64_t j = 0; j < F; ++j) acc += (e4m3_value(q2[i * F + j]) * sc2) * (e4m3_value(h8[j]) * (double)hs);
+        o[i] = acc;
+    }
+}
+
+static void forward_fp8_range(void* p, int64_t b, int64_t e) {
+    fwd8_ctx* c = (fwd8_ctx*)p;
+    const int64_t d = c->d, F = c->F;
+    double* xd = (double*)malloc(sizeof(double) * (size_t)d);
+    uint8_t* xq = (uint8_t*)malloc((size_t)d);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    uint8_t* h8 = (uint8_t*)malloc((size_t)F);
+    double* o = (double*)malloc(sizeof(double) * (size_t)d);
+    int32_t ids[64];
+    double wts[64];
+    for (int64_t n = b; n < e; ++n) {
+        const int64_t t = c->tokens ? c->tokens[n] : n;
+        const uint16_t* xt = c->x + t * d;
+        float xs;
+        quantize_row_fp8(xt, d, xq, &xs); /* per-token activation scale */
+        for (int64_t i = 0; i < d; ++i) xd[i] = e4m3_value(xq[i]) * (double)xs;
+        route_token(xt, d, c->wr, c->bias, c->E, c->K, ids, wts, NULL); /* the router sees the bf16 x */
+        double* yt = c->y + n * d;
+        for (int64_t i = 0; i < d; ++i) yt[i] = 0.0;
+        for (int k = 0; k < c->K; ++k) {
+            expert_ffn_fp8(c, ids[k], xd, h, h8, o);
+            for (int64_t i = 0; i < d; ++i) yt[i] += wts[k] * o[i];
+            if (c->h_out) memcpy(c->h_out + (n * c->K + k) * F, h, sizeof(double) * (size_t)F);
+            if (c->ids) c->ids[n * c->K + k] = ids[k];
+            if (c->wts) c->wts[n * c->K + k] = wts[k];
+        }
+    }
+    free(xd);
+    free(xq);
+    free(h);
+    free(h8);
+    free(o);
+}
+
+/* The FP8 layer on a subset of tokens; arguments as oracle_moe_forward with E4M3 codes for q1, q3, q2
+ * (scales from oracle_quantize_rows_fp8); h_out gets the SwiGLU intermediate before its quantization. */
+int oracle_moe_forward_fp8(const uint16_t* x, int64_t T, int64_t d, int64_t F, int E, int K, const float* wr,
+                           const float* bias, const uint8_t* q1, const float* s1, const uint8_t* q3, const float* s3,
+                           const uint8_t* q2, const float* s2, const int64_t* tokens, int64_t n_tokens, double* y,
+                           int32_t* ids, double* wts, double* h_out, int threads) {
+    if (!x || !wr || !q1 || !s1 || !q3 || !s3 || !q2 || !s2 || !y) return -1;
+    if (T < 0 || d <= 0 || F <= 0 || E < 1 || E > 64 || K < 1 || K > E || n_tokens < 0) return -1;
+    if (tokens) {
+        for (int64_t n = 0; n < n_tokens; ++n)
+            if (tokens[n] < 0 || tokens[n] >= T) return -1;
+    } else if (n_tokens > T) {
+        return -1;
+    }
+    fwd8_ctx c = {x, d, F, E, K, wr, bias, q1, q3, q2, s1, s3, s2, tokens, y, ids, wts, h_out};
+    parallel_for(n_tokens, threads, forward_fp8_range, &c);
     return 0;
 }
 

@@ -368,4 +368,121 @@ def pin_mlp_one_hot_and_token_subset(orc):
     assert np.allclose(out["h"][0], torch.nn.functional.silu(a1).numpy() * a3, rtol=1e-14, atol=0)
 
 
+# ------------------------------------------------------------- FP8 (E4M3) layer
+
+
+def torch_e4m3(v):
+    """torch's own float8_e4m3fn cast (nearest, ties to even; no saturation: |v| must be < 464)."""
+    t = torch.as_tensor(np.asarray(v, dtype=np.float32)).to(torch.float8_e4m3fn)
+    return t.view(torch.uint8).numpy(), t.to(torch.float64).numpy()
+
+
+E4M3_VALUES = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def pin_e4m3_rounding_against_torch(orc):
+    rng = np.random.default_rng(41)
+    finite = E4M3_VALUES[np.isfinite(E4M3_VALUES)]
+    pos = np.unique(finite[finite >= 0])
+    mids = (pos[1:] + pos[:-1]) / 2  # every tie, between every pair of neighbours
+    v = np.concatenate([rng.standard_normal(20000) * 30, rng.standard_normal(4000) * 1e-2,
+                        rng.uniform(-2e-3, 2e-3, 2000), mids, -mids, pos, -pos, [447.9, -447.9, 1e-30]])
+    v = v.astype(np.float32).astype(np.float64)  # exact in fp32, so torch's cast rounds once
+    codes, vals = orc.e4m3_round(v)
+    tc, tv = torch_e4m3(v)
+    assert np.array_equal(codes, tc)
+    assert np.array_equal(vals, tv)
+    # saturation (torch gives NaN there): +-448
+    c2, v2 = orc.e4m3_round(np.array([448.0, 463.9, 464.0, 1e6, -500.0]))
+    assert v2.tolist() == [448.0, 448.0, 448.0, 448.0, -448.0] and c2.tolist() == [0x7E] * 4 + [0xFE]
+
+
+def pin_quantize_fp8_exact_rational(orc):
+    rng = np.random.default_rng(42)
+    w = random_bf16(rng, (10, 48), 0.02)
+    w[2, 5] = bf16_bits([0.90625])[0]
+    w[4] = 0
+    q, s = orc.quantize_fp8(w)
+    finite = np.isfinite(E4M3_VALUES)
+    table = [(Fraction(float(E4M3_VALUES[c])), c) for c in range(256) if finite[c]]
+    for r in range(w.shape[0]):
+        vals = [Fraction(float(v)) for v in synth.bf16_bits_to_f32(w[r])]
+        amax = max(abs(v) for v in vals)
+        if amax == 0:
+            assert s[r] == 1.0 and not q[r].any()
+            continue
+        scale = f32_nearest(amax / 448)
+        assert float(s[r]) == scale
+        for i, v in enumerate(vals):
+            quot = v / Fraction(scale)
+            best = min(abs(quot - tv) for tv, _ in table)
+            cands = sorted({c for tv, c in table if abs(quot - tv) == best and not (tv == 0 and c == 0x80)})
+            if len(cands) > 1:  # a tie: the even code (zero is +0 unless the value is negative zero)
+                cands = [c for c in cands if c % 2 == 0]
+            assert q[r, i] == cands[0] or (quot == 0 and q[r, i] in (0, 0x80)), (r, i)
+
+
+def fp8_layer(rng, T=6, d=32, F=40, E=16):
+    """Random FP8 codes (finite) and scales for a small layer, built directly."""
+    finite = np.flatnonzero(np.isfinite(E4M3_VALUES)).astype(np.uint8)
+    L = tiny_layer(rng, T=T, d=d, F=F, E=E)
+    for k in ("q1", "q3", "q2"):
+        L[k] = rng.choice(finite, size=L[k].shape).astype(np.uint8)
+    for k in ("s1", "s3", "s2"):
+        L[k] = (L[k] * np.float32(127 / 448 / 8)).astype(np.float32)
+    return L
+
+
+def torch_fp8_ffn(xf, q1, s1, q3, s3, q2, s2):
+    """One FP8 expert on every row of xf with torch's float8 cast for the activations and h:
+    per-row scales amax / 448 in fp32."""
+    def quant_rows(a):
+        amax = np.abs(a).max(axis=1).astype(np.float32)
+        sc = np.where(amax == 0, np.float32(1), amax / np.float32(448)).astype(np.float32)
+        _, v = torch_e4m3((a / sc[:, None].astype(np.float64)).astype(np.float32))
+        return v * sc[:, None].astype(np.float64)
+    w = lambda q, s: E4M3_VALUES[q] * s.astype(np.float64)[:, None]  # noqa: E731
+    xd = quant_rows(xf)
+    a1, a3 = xd @ w(q1, s1).T, xd @ w(q3, s3).T
+    h = torch.nn.functional.silu(torch.as_tensor(a1)).numpy() * a3
+    return quant_rows(h) @ w(q2, s2).T, h
+
+
+def pin_fp8_forward_against_torch_float8(orc):
+    # every expert on every token with torch's float8 casts and matmul, gated by numpy top-2
+    rng = np.random.default_rng(43)
+    L = fp8_layer(rng, T=7, d=32, F=48)
+    out = orc.moe_forward_fp8(L["x"], L["wr"], None, L["q1"], L["s1"], L["q3"], L["s3"], L["q2"], L["s2"],
+                              want_hidden=True)
+    xf = synth.bf16_bits_to_f32(L["x"]).astype(np.float64)
+    z = xf @ L["wr"].astype(np.float64).T
+    p = torch.softmax(torch.as_tensor(z), 1).numpy()
+    top = np.argsort(-z, axis=1, kind="stable")[:, :2]
+    y_ref = np.zeros_like(xf)
+    for e in range(16):
+        ye, he = torch_fp8_ffn(xf, L["q1"][e], L["s1"][e], L["q3"][e], L["s3"][e], L["q2"][e], L["s2"][e])
+        y_ref += np.where((top == e).any(1), p[:, e], 0.0)[:, None] * ye
+        for k in range(2):
+            sel = top[:, k] == e
+            assert np.allclose(out["h"][sel, k], he[sel], rtol=1e-12, atol=1e-15)
+    assert np.array_equal(out["ids"], top)
+    assert np.allclose(out["y"], y_ref, rtol=1e-10, atol=1e-13)
+
+
+def pin_fp8_forward_zero_gate_and_exact_grid(orc):
+    rng = np.random.default_rng(44)
+    L = fp8_layer(rng)
+    M = dict(L)
+    M["q1"] = np.zeros_like(L["q1"])
+    out = orc.moe_forward_fp8(M["x"], M["wr"], None, M["q1"], M["s1"], M["q3"], M["s3"], M["q2"], M["s2"])
+    assert not np.any(out["y"])
+    # activations already on the E4M3 grid with amax 448 * 2^-6: quantizing them is exact
+    vals = E4M3_VALUES[np.isfinite(E4M3_VALUES)]
+    x = rng.choice(vals[np.abs(vals) <= 448], size=(3, 32)) * 2.0 ** -6
+    x[:, 0] = 448 * 2.0 ** -6
+    L["x"] = bf16_bits(x.astype(np.float32))
+    q, sx = orc.quantize_fp8(L["x"])
+    assert np.all(sx == np.float32(2.0 ** -6)) and np.array_equal(E4M3_VALUES[q] * 2.0 ** -6, x)
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -32,6 +32,11 @@ MUTANTS = {
                                "n : n;\n        const uint16_t* xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn"),
     "mlp_first_token_only": ("xt = c->x + t * d;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn",
                              "xt = c->x;\n        for (int64_t i = 0; i < d; ++i) xd[i] = (double)bf16_value(xt[i]);\n        expert_ffn"),
+    "fp8_scale_over_512": ("amax / 448.0f", "amax / 512.0f"),
+    "fp8_ties_away": ("nearbyint(ldexp(a, 3 - eb))", "round(ldexp(a, 3 - eb))"),
+    "fp8_flush_subnormals": ("if (eb < -6) eb = -6;", "if (eb < -6) return sign;"),
+    "fp8_h_not_quantized": ("(e4m3_value(h8[j]) * (double)hs)", "h[j]"),
+    "fp8_x_not_quantized": ("xd[i] = e4m3_value(xq[i]) * (double)xs;", "xd[i] = (double)bf16_value(xt[i]);"),
     "router_ignores_last_input": ("for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i])",
                                   "for (int64_t i = 0; i + 1 < d; ++i) acc += (double)bf16_value(x[i])"),
 }
