@@ -541,10 +541,21 @@ typedef struct {
     double* h_out;
 } fwd8_ctx;
 
+/* fp32 -> bf16, round to nearest even (finite values). */
+static double bf16_round(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+    float r;
+    memcpy(&r, &u, 4);
+    return (double)r;
+}
+
 /* One FP8 expert on one token whose activations xd are already the dequantized E4M3 values:
  *   a1_j = sum_i (v(q1[j][i]) s1_j) xd_i, a3_j likewise, h_j = SiLU(a1_j) a3_j,
- *   h quantized per row (scale = fp32(amax_j |h_j|) / 448 in fp32, codes of h_j / scale),
- *   o_i = sum_j (v(q2[i][j]) s2_i) hd_j with hd the dequantized h. */
+ *   h held in bf16 between the two GEMMs, as in the ExpertsInt8 layer (fp64 -> fp32 -> bf16, each
+ *   to nearest even), then quantized per row (scale = amax_j |h_j| / 448 in fp32, codes of
+ *   h_j / scale), o_i = sum_j (v(q2[i][j]) s2_i) hd_j with hd the dequantized h. */
 static void expert_ffn_fp8(const fwd8_ctx* c, int e, const double* xd, double* h, uint8_t* h8, double* o) {
     const int64_t d = c->d, F = c->F;
     const uint8_t* q1 = c->q1 + (int64_t)e * F * d;
@@ -562,10 +573,11 @@ static void expert_ffn_fp8(const fwd8_ctx* c, int e, const double* xd, double* h
             a3 += (e4m3_value(q3[j * d + i]) * sc3) * xd[i];
         }
         h[j] = a1 / (1.0 + exp(-a1)) * a3;
-        if (fabs(h[j]) > amax) amax = fabs(h[j]);
+        const double hb = bf16_round((float)h[j]);
+        if (fabs(hb) > amax) amax = fabs(hb);
     }
     const float hs = (amax == 0.0) ? 1.0f : (float)amax / 448.0f;
-    for (int64_t j = 0; j < F; ++j) h8[j] = (amax == 0.0) ? 0 : e4m3_round(h[j] / (double)hs);
+    for (int64_t j = 0; j < F; ++j) h8[j] = (amax == 0.0) ? 0 : e4m3_round(bf16_round((float)h[j]) / (double)hs);
     for (int64_t i = 0; i < d; ++i) {
         double acc = 0.0;
         const double sc2 = (double)s2[i];

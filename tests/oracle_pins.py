@@ -434,8 +434,8 @@ def fp8_layer(rng, T=6, d=32, F=40, E=16):
 
 
 def torch_fp8_ffn(xf, q1, s1, q3, s3, q2, s2):
-    """One FP8 expert on every row of xf with torch's float8 cast for the activations and h:
-    per-row scales amax / 448 in fp32."""
+    """One FP8 expert on every row of xf with torch's float8 cast for the activations and for h
+    (held in bf16 first, torch's casts): per-row scales amax / 448 in fp32."""
     def quant_rows(a):
         amax = np.abs(a).max(axis=1).astype(np.float32)
         sc = np.where(amax == 0, np.float32(1), amax / np.float32(448)).astype(np.float32)
@@ -445,7 +445,8 @@ def torch_fp8_ffn(xf, q1, s1, q3, s3, q2, s2):
     xd = quant_rows(xf)
     a1, a3 = xd @ w(q1, s1).T, xd @ w(q3, s3).T
     h = torch.nn.functional.silu(torch.as_tensor(a1)).numpy() * a3
-    return quant_rows(h) @ w(q2, s2).T, h
+    hb = torch.as_tensor(h).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()  # h held in bf16
+    return quant_rows(hb) @ w(q2, s2).T, h
 
 
 def pin_fp8_forward_against_torch_float8(orc):

@@ -36,6 +36,7 @@ MUTANTS = {
     "fp8_ties_away": ("nearbyint(ldexp(a, 3 - eb))", "round(ldexp(a, 3 - eb))"),
     "fp8_flush_subnormals": ("if (eb < -6) eb = -6;", "if (eb < -6) return sign;"),
     "fp8_h_not_quantized": ("(e4m3_value(h8[j]) * (double)hs)", "h[j]"),
+    "fp8_h_not_bf16": ("e4m3_round(bf16_round((float)h[j]) / (double)hs)", "e4m3_round(h[j] / (double)hs)"),
     "fp8_x_not_quantized": ("xd[i] = e4m3_value(xq[i]) * (double)xs;", "xd[i] = (double)bf16_value(xt[i]);"),
     "router_ignores_last_input": ("for (int64_t i = 0; i < d; ++i) acc += (double)bf16_value(x[i])",
                                   "for (int64_t i = 0; i + 1 < d; ++i) acc += (double)bf16_value(x[i])"),
