@@ -42,8 +42,9 @@ def parse():
                     help="MoE layer workloads, or mlp_* for the dense ExpertsInt8 MLP")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
-    ap.add_argument("--weights", default="int8", choices=["int8", "bf16"],
-                    help="int8: ExpertsInt8 (the method); bf16: the unquantized comparator layer")
+    ap.add_argument("--weights", default="int8", choices=["int8", "bf16", "fp8"],
+                    help="int8: ExpertsInt8 (the method); bf16: the unquantized comparator layer; "
+                         "fp8: the FP8 (E4M3 weights and activations) comparator layer")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
@@ -90,6 +91,8 @@ def algorithmic(kind, wl, T, touched, rows_padded, wbytes=1):
         return "bytes", rows_padded * d * 2 + TK * d * 2
     if kind == "permute":
         return "bytes", TK * 4 * 3
+    if kind == "act_quant":  # FP8 layer, per launch on average: x (bf16 -> E4M3) and h (fp32 -> E4M3)
+        return "bytes", (T * d * 3 + TK * F * 5) / 2
     if kind == "quantize":
         return "bytes", 3 * (2 * F * d + d * F) * wl.E
     return "bytes", 0
@@ -331,7 +334,8 @@ def run_ours(args):
     bias_np = synth.gen_bias(wl)
     bias = None if bias_np is None else torch.from_numpy(bias_np).to(dev)
     int8w = args.weights == "int8"
-    wbytes = 1 if int8w else 2
+    fp8 = args.weights == "fp8"
+    wbytes = 2 if args.weights == "bf16" else 1
     Q, S, Wb = {}, {}, {}
     q_ms = 0.0
     jm.jamba_moe_timing_start(3)  # the quantize launches (one per matrix), timed by the library's own events
@@ -343,11 +347,15 @@ def run_ours(args):
         if int8w:
             Q[which], S[which] = jm.jamba_moe_quantize(Wb[which])
             del Wb[which]
+        elif fp8:
+            Q[which], S[which] = jm.jamba_moe_quantize_fp8(Wb[which])
+            del Wb[which]
     torch.cuda.synchronize()
     q_ms = jm.jamba_moe_timing_collect().get("quantize", (0.0, 0))[0]
     jm.jamba_moe_timing_start(0)
     q_bytes = algorithmic("quantize", wl, T, 0, 0)[1]
-    ws_bytes = jm.jamba_mlp_workspace_size(T, d, F) if mlp else jm.jamba_moe_workspace_size(T, d, F)
+    ws_bytes = (jm.jamba_mlp_workspace_size(T, d, F) if mlp else
+                jm.jamba_moe_workspace_size_fp8(T, d, F) if fp8 else jm.jamba_moe_workspace_size(T, d, F))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     y = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
     ids = torch.empty((T, 2), dtype=torch.int32, device=dev)
@@ -361,6 +369,9 @@ def run_ours(args):
         elif int8w:
             jm.jamba_moe_forward(xin, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
                                  topk_ids=ids, topk_w=tw, workspace=ws, path=path)
+        elif fp8:
+            jm.jamba_moe_forward_fp8(xin, wr, bias, Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"], y=y,
+                                     topk_ids=ids, topk_w=tw, workspace=ws, path=path)
         else:
             jm.jamba_moe_forward_bf16w(xin, wr, bias, Wb["w1"], Wb["w3"], Wb["w2"], y=y, topk_ids=ids, topk_w=tw,
                                        workspace=ws, path=path)
@@ -429,10 +440,14 @@ def run_ours(args):
     if unit_kind == "bytes":
         achieved, peak, unit, bound = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
     else:
-        achieved, peak, unit, bound = work / avg_s / 1e12, peaks["bf16_tflops_sustained"], "TFLOP/s", "tensor"
+        # FP8 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        achieved, peak, unit, bound = (work / avg_s / 1e12, peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0),
+                                       "TFLOP/s", "tensor")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                "traffic": ncu_traffic(dom, wl.name), "kernel": dom, "algorithmic_per_launch": work,
-                "peak_source": peaks["source"]}
+                "traffic": ncu_traffic(dom, wl.name) if args.weights == "int8" else None, "kernel": dom,
+                "algorithmic_per_launch": work,
+                "peak_source": peaks["source"] + (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 and bound == "tensor"
+                                                  else "")}
     per_kernel = {}
     for k, (kms, n) in sorted(kernels.items(), key=lambda kv: -kv[1][0]):
         uk, wk = algorithmic(k, wl, T, touched, rows_padded, wbytes)
@@ -454,8 +469,10 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
-                           weights=("int8 codes + fp32 per-output-channel scales" if int8w
-                                    else "bf16 (unquantized comparator)")),
+                           weights=("int8 codes + fp32 per-output-channel scales" if int8w else
+                                    "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
+                                    "per-row scales (FP8 comparator)" if fp8 else
+                                    "bf16 (unquantized comparator)")),
             "roofline": roofline, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 2},

@@ -136,6 +136,40 @@ int jamba_moe_forward_bf16w(const uint16_t* x, const float* router_W, const floa
                             void* workspace, size_t workspace_bytes, void* stream, int path);
 
 /*
+ * FP8 comparator layer.  The Jamba-1.5 paper (§3.1) compares ExpertsInt8 with FP8 serving (on H100,
+ * ExpertsInt8 matches FP8's latency; FP8 needs FP8 hardware and, unlike ExpertsInt8, does not keep
+ * BF16 activations) without defining the FP8 scheme.  This library's reading: both GEMM operands
+ * are OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+ * finite 448, subnormals m * 2^-9); weights carry one fp32 scale per output channel, the
+ * activations x one dynamic fp32 scale per token and the SwiGLU intermediate one per expert row
+ * (scale = amax / 448 in fp32, code = the E4M3 value nearest to the exact quotient, ties to the
+ * even code, saturating at +-448; a row of zeros gets scale 1).  Router and combine as in
+ * jamba_moe_forward.
+ *
+ * jamba_moe_quantize_fp8 — as jamba_moe_quantize with E4M3 codes: Q uint8 [n_mats][rows][cols].
+ * Bit-exact and deterministic.
+ */
+int jamba_moe_quantize_fp8(const uint16_t* W, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* Q, float* S,
+                           void* stream);
+
+/* jamba_moe_workspace_size_fp8 — device scratch bytes of jamba_moe_forward_fp8 (0: unsupported sizes). */
+size_t jamba_moe_workspace_size_fp8(int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k);
+
+/*
+ * jamba_moe_forward_fp8 — the FP8 layer: arguments as jamba_moe_forward_path, with Q1, Q3
+ * uint8 [n_experts][ffn][d] and Q2 uint8 [n_experts][d][ffn] E4M3 codes from
+ * jamba_moe_quantize_fp8 and their scales.  x is quantized per token, the fp32 SwiGLU output of
+ * the first GEMM per expert row; the GEMMs multiply E4M3 by E4M3 with fp32 accumulation (tcgen05
+ * kind::f8f6f4 on the tensor-core path, mma.sync e4m3 on the decode path) and apply the weight and
+ * activation scales to the fp32 totals.  Deterministic; errors as jamba_moe_forward.
+ */
+int jamba_moe_forward_fp8(const uint16_t* x, const float* router_W, const float* router_bias, const uint8_t* Q1,
+                          const float* S1, const uint8_t* Q3, const float* S3, const uint8_t* Q2, const float* S2,
+                          int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y,
+                          int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes, void* stream,
+                          int path);
+
+/*
  * jamba_mlp_workspace_size — bytes of device scratch jamba_mlp_forward needs for these sizes.
  * Returns 0 for unsupported sizes.  Host only; touches no device.
  */
@@ -236,7 +270,8 @@ enum {
     JMOE_KERNEL_GEMM13 = 6,
     JMOE_KERNEL_GEMM2 = 7,
     JMOE_KERNEL_COMBINE = 8,
-    JMOE_KERNEL_KINDS = 9
+    JMOE_KERNEL_ACT_QUANT = 9, /* FP8 layer: per-row E4M3 quantization of x and of the intermediate h */
+    JMOE_KERNEL_KINDS = 10
 };
 int jamba_moe_timing_start(int max_launches);
 int jamba_moe_timing_collect(double* total_ms, int64_t* launches, int n_kinds);

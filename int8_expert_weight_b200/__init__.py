@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(HERE, "libjmoe.so")
 N_EXPERTS = 16
 TOP_K = 2
 PATH_AUTO, PATH_GEMV, PATH_GEMM = 0, 1, 2
-KERNEL_NAMES = ["quantize", "router", "permute", "gather", "gemv13", "gemv2", "gemm13", "gemm2", "combine"]
+KERNEL_NAMES = ["quantize", "router", "permute", "gather", "gemv13", "gemv2", "gemm13", "gemm2", "combine",
+                "act_quant"]
 
 
 class JmoeError(RuntimeError):
@@ -48,6 +49,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_workspace_size.argtypes = [i64, i64, i64, c_int, c_int]
     fwd_args = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, sz, vp]
     lib.jamba_moe_forward.restype = c_int
+    lib.jamba_moe_quantize_fp8.restype = c_int
+    lib.jamba_moe_quantize_fp8.argtypes = [vp, i64, i64, i64, vp, vp, vp]
+    lib.jamba_moe_workspace_size_fp8.restype = sz
+    lib.jamba_moe_workspace_size_fp8.argtypes = [i64, i64, i64, c_int, c_int]
+    lib.jamba_moe_forward_fp8.restype = c_int
+    lib.jamba_moe_forward_fp8.argtypes = fwd_args + [c_int]
     lib.jamba_mlp_workspace_size.restype = sz
     lib.jamba_mlp_workspace_size.argtypes = [i64, i64, i64]
     mlp_args = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]
@@ -186,6 +193,82 @@ def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Opti
                                     workspace.data_ptr(), workspace.numel(), _stream_ptr(stream), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward")
+    return y, topk_ids, topk_w
+
+
+def jamba_moe_quantize_fp8(W: torch.Tensor, stream: Optional[torch.cuda.Stream] = None,
+                           out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """FP8 (E4M3) quantization of bf16 weights [..., rows, cols] (one scale per row).
+    Returns (Q uint8 E4M3 codes, same shape; S fp32, shape[:-1])."""
+    lib = load_library()
+    _check(W, "W", torch.bfloat16)
+    if W.dim() < 2:
+        raise ValueError("W must have at least 2 dims (rows, cols)")
+    rows, cols = W.shape[-2], W.shape[-1]
+    n_mats = W.numel() // (rows * cols) if W.numel() else 0
+    if out is None:
+        Q = torch.empty(W.shape, dtype=torch.uint8, device=W.device)
+        S = torch.empty(W.shape[:-1], dtype=torch.float32, device=W.device)
+    else:
+        Q, S = out
+        _check(Q, "Q", torch.uint8, W.shape)
+        _check(S, "S", torch.float32, W.shape[:-1])
+    st = lib.jamba_moe_quantize_fp8(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(), _stream_ptr(stream))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_quantize_fp8")
+    return Q, S
+
+
+def jamba_moe_workspace_size_fp8(T: int, d: int, ffn: int, n_experts: int = N_EXPERTS, top_k: int = TOP_K) -> int:
+    return int(load_library().jamba_moe_workspace_size_fp8(T, d, ffn, n_experts, top_k))
+
+
+def jamba_moe_forward_fp8(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor],
+                          Q1: torch.Tensor, S1: torch.Tensor, Q3: torch.Tensor, S3: torch.Tensor,
+                          Q2: torch.Tensor, S2: torch.Tensor, y: Optional[torch.Tensor] = None,
+                          topk_ids: Optional[torch.Tensor] = None, topk_w: Optional[torch.Tensor] = None,
+                          workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None,
+                          path: int = PATH_AUTO):
+    """The FP8 (E4M3) comparator layer: as jamba_moe_forward with uint8 E4M3 codes Q1, Q3, Q2 from
+    jamba_moe_quantize_fp8.  Returns (y, topk_ids, topk_w)."""
+    lib = load_library()
+    _check(x, "x", torch.bfloat16)
+    if x.dim() != 2:
+        raise ValueError("x must be [T][d]")
+    T, d = x.shape
+    E = router_W.shape[0]
+    ffn = Q1.shape[1]
+    _check(router_W, "router_W", torch.float32, (E, d))
+    if router_bias is not None:
+        _check(router_bias, "router_bias", torch.float32, (E,))
+    _check(Q1, "Q1", torch.uint8, (E, ffn, d))
+    _check(Q3, "Q3", torch.uint8, (E, ffn, d))
+    _check(Q2, "Q2", torch.uint8, (E, d, ffn))
+    _check(S1, "S1", torch.float32, (E, ffn))
+    _check(S3, "S3", torch.float32, (E, ffn))
+    _check(S2, "S2", torch.float32, (E, d))
+    if y is None:
+        y = torch.empty((T, d), dtype=torch.bfloat16, device=x.device)
+    _check(y, "y", torch.bfloat16, (T, d))
+    if topk_ids is None:
+        topk_ids = torch.empty((T, TOP_K), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, TOP_K), dtype=torch.float32, device=x.device)
+    _check(topk_ids, "topk_ids", torch.int32, (T, TOP_K))
+    _check(topk_w, "topk_w", torch.float32, (T, TOP_K))
+    need = jamba_moe_workspace_size_fp8(T, d, ffn, E, TOP_K)
+    if need == 0:
+        raise JmoeError(2, "jamba_moe_workspace_size_fp8")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    _check(workspace, "workspace", torch.uint8)
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    st = lib.jamba_moe_forward_fp8(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(), S1.data_ptr(),
+                                   Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(), T, d, ffn, E, TOP_K,
+                                   y.data_ptr(), p(topk_ids), p(topk_w), workspace.data_ptr(), workspace.numel(),
+                                   _stream_ptr(stream), int(path))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_forward_fp8")
     return y, topk_ids, topk_w
 
 

@@ -45,6 +45,21 @@ cudaError_t launch_gemv2_dense(const WsHeader* hdr, const int32_t* perm, const u
                                const float* S2, const float* wts, uint16_t* y, int64_t T, int64_t d, int64_t F,
                                cudaStream_t st);
 
+cudaError_t launch_quantize_fp8(const uint16_t* W, int64_t rows, int64_t cols, uint8_t* Q, float* S,
+                                const int32_t* perm, const int32_t* n_live, cudaStream_t st, int num_sms);
+cudaError_t launch_gemv13_f8(const WsHeader* hdr, const int32_t* perm, const uint8_t* x8, const float* sx,
+                             const uint8_t* Q1, const float* S1, const uint8_t* Q3, const float* S3, uint16_t* h,
+                             int64_t T, int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemv2_f8(const WsHeader* hdr, const int32_t* perm, const uint8_t* h8, const float* sh,
+                            const uint8_t* Q2, const float* S2, const float* wts, float* out_slot, int64_t T,
+                            int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemm13_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* x8_perm, const float* sx,
+                             const uint8_t* Q1, const float* S1, const uint8_t* Q3, const float* S3, uint16_t* h,
+                             int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st);
+cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h8, const float* sh, const uint8_t* Q2,
+                            const float* S2, const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F,
+                            cudaStream_t st);
+
 namespace {
 
 constexpr int64_t kMaxT = int64_t(1) << 20;
@@ -331,6 +346,164 @@ int mlp_impl(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t*
 
 }  // namespace
 
+namespace {
+
+// ---------------------------------------------------------------- FP8 (E4M3) comparator layer
+struct LayoutF8 {
+    int64_t rows_cap;
+    size_t hdr, ids, wts, inv, perm, x8, sx, x8_perm, h, h8, sh, slots, total;
+};
+
+LayoutF8 make_layout_f8(int64_t T, int64_t d, int64_t F) {
+    LayoutF8 L{};
+    const int64_t TK = T * kTopK;
+    L.rows_cap = (TK + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.hdr = take(kHeaderBytes);
+    L.ids = take(sizeof(int32_t) * TK);
+    L.wts = take(sizeof(float) * TK);
+    L.inv = take(sizeof(int32_t) * TK);
+    L.perm = take(sizeof(int32_t) * L.rows_cap);
+    L.x8 = take((size_t)T * d);
+    L.sx = take(sizeof(float) * T);
+    L.x8_perm = take((size_t)L.rows_cap * d);
+    L.h = take(sizeof(uint16_t) * L.rows_cap * F);
+    L.h8 = take((size_t)L.rows_cap * F);
+    L.sh = take(sizeof(float) * L.rows_cap);
+    L.slots = take(sizeof(float) * TK * d);
+    L.total = off;
+    return L;
+}
+
+int forward_f8(const uint16_t* x, const float* router_W, const float* router_bias, const uint8_t* Q1, const float* S1,
+               const uint8_t* Q3, const float* S3, const uint8_t* Q2, const float* S2, int64_t T, int64_t d,
+               int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w, void* workspace,
+               size_t workspace_bytes, void* stream, int path) {
+    if (!x || !router_W || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
+    if (!shape_ok(T, d, ffn, n_experts, top_k)) return JMOE_ERR_SHAPE;
+    if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    const void* ptrs16[] = {x, Q1, Q3, Q2, y, router_W};
+    for (const void* p : ptrs16)
+        if (!aligned16(p)) return JMOE_ERR_ALIGN;
+    const void* ptrs4[] = {router_bias, S1, S3, S2, topk_ids, topk_w};
+    for (const void* p : ptrs4)
+        if (reinterpret_cast<uintptr_t>(p) & 3) return JMOE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return JMOE_ERR_WORKSPACE;
+    const LayoutF8 L = make_layout_f8(T, d, ffn);
+    if (workspace_bytes < L.total) return JMOE_ERR_WORKSPACE;
+
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+    int32_t* ids = reinterpret_cast<int32_t*>(ws + L.ids);
+    float* wts = reinterpret_cast<float*>(ws + L.wts);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    uint8_t* x8 = reinterpret_cast<uint8_t*>(ws + L.x8);
+    float* sx = reinterpret_cast<float*>(ws + L.sx);
+    uint8_t* x8_perm = reinterpret_cast<uint8_t*>(ws + L.x8_perm);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    uint8_t* h8 = reinterpret_cast<uint8_t*>(ws + L.h8);
+    float* sh = reinterpret_cast<float*>(ws + L.sh);
+    float* slots = reinterpret_cast<float*>(ws + L.slots);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = num_sms_current();
+    if (path == JMOE_PATH_AUTO) path = (T <= kGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
+
+    cudaError_t e;
+    {
+        TimedLaunch t(JMOE_KERNEL_ROUTER, st);
+        e = launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
+        e = launch_permute(ids, T, hdr, perm, inv, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_ACT_QUANT, st);  // per-token E4M3 activations
+        e = launch_quantize_fp8(x, T, d, x8, sx, nullptr, nullptr, st, sms);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    const int32_t* n_rows = &hdr->seg_start[kExperts];
+    if (path == JMOE_PATH_GEMV) {
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV13, st);
+            e = launch_gemv13_f8(hdr, perm, x8, sx, Q1, S1, Q3, S3, h, T, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_ACT_QUANT, st);  // per-row E4M3 intermediate
+            e = launch_quantize_fp8(h, L.rows_cap, ffn, h8, sh, perm, n_rows, st, sms);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV2, st);
+            e = launch_gemv2_f8(hdr, perm, h8, sh, Q2, S2, wts, slots, T, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    } else {
+        {
+            TimedLaunch t(JMOE_KERNEL_GATHER, st);  // E4M3 rows, moved as pairs of bytes
+            e = launch_gather(reinterpret_cast<const uint16_t*>(x8), perm, hdr, d / 2, L.rows_cap,
+                              reinterpret_cast<uint16_t*>(x8_perm), st, sms, false);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMM13, st);
+            e = launch_gemm13_f8(hdr, perm, x8_perm, sx, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_ACT_QUANT, st);
+            e = launch_quantize_fp8(h, L.rows_cap, ffn, h8, sh, perm, n_rows, st, sms);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMM2, st);
+            e = launch_gemm2_f8(hdr, perm, h8, sh, Q2, S2, wts, slots, L.rows_cap, d, ffn, st);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    }
+    TimedLaunch t(JMOE_KERNEL_COMBINE, st);
+    return to_status(launch_combine(slots, T, d, y, st, sms));
+}
+
+}  // namespace
+
+extern "C" {
+
+int jamba_moe_quantize_fp8(const uint16_t* W, int64_t n_mats, int64_t rows, int64_t cols, uint8_t* Q, float* S,
+                           void* stream) {
+    if (!W || !Q || !S) return JMOE_ERR_NULL;
+    if (n_mats < 1 || rows < 1 || cols < 16 || cols > (int64_t(1) << 20) || cols % 16 != 0) return JMOE_ERR_SHAPE;
+    if (n_mats > (int64_t(1) << 40) / rows) return JMOE_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(Q) || (reinterpret_cast<uintptr_t>(S) & 3)) return JMOE_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TimedLaunch t(JMOE_KERNEL_QUANTIZE, st);
+    return to_status(launch_quantize_fp8(W, n_mats * rows, cols, Q, S, nullptr, nullptr, st, num_sms_current()));
+}
+
+size_t jamba_moe_workspace_size_fp8(int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k) {
+    if (!shape_ok(T, d, ffn, n_experts, top_k)) return 0;
+    return make_layout_f8(T, d, ffn).total;
+}
+
+int jamba_moe_forward_fp8(const uint16_t* x, const float* router_W, const float* router_bias, const uint8_t* Q1,
+                          const float* S1, const uint8_t* Q3, const float* S3, const uint8_t* Q2, const float* S2,
+                          int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids,
+                          float* topk_w, void* workspace, size_t workspace_bytes, void* stream, int path) {
+    return forward_f8(x, router_W, router_bias, Q1, S1, Q3, S3, Q2, S2, T, d, ffn, n_experts, top_k, y, topk_ids,
+                      topk_w, workspace, workspace_bytes, stream, path);
+}
+
+}  // extern "C"
+
 extern "C" {
 
 size_t jamba_mlp_workspace_size(int64_t T, int64_t d, int64_t ffn) {
@@ -444,7 +617,7 @@ int jamba_moe_timing_collect(double* total_ms, int64_t* launches, int n_kinds) {
 
 const char* jamba_moe_kernel_name(int kind) {
     static const char* names[JMOE_KERNEL_KINDS] = {"quantize", "router", "permute", "gather", "gemv13",
-                                                   "gemv2", "gemm13", "gemm2", "combine"};
+                                                   "gemv2", "gemm13", "gemm2", "combine", "act_quant"};
     return (kind >= 0 && kind < JMOE_KERNEL_KINDS) ? names[kind] : "unknown";
 }
 

@@ -49,6 +49,9 @@ struct GemmArgs {
     uint32_t max_polls;   // bound of every mbarrier wait
     int skip_copy;        // test hook: CTA 0 skips the copies of its second K step (a wait then runs out)
     uint16_t* y_out;      // gemm2 of the dense MLP: y [T][N] in bf16, written instead of out_slot
+    // FP8 layer only: per-row activation scale (gemm13: per token, indexed by assignment / K;
+    // gemm2: per permuted row)
+    const float* a_scale;
 };
 
 // Shared-memory ring: per stage the activation tile, the bf16 weight tile the MMA reads and, for
@@ -113,7 +116,9 @@ __device__ __forceinline__ bool tile_coord(const WsHeader* hdr, const GemmArgs& 
     return false;
 }
 
-template <bool kDual, int BN, bool kW8>
+// kF8: both operands E4M3 codes copied by TMA into the MMA's layout (no conversion), 128 K
+// elements (128 bytes) per stage, kind::f8f6f4 MMAs, activation and weight scales in the epilogue.
+template <bool kDual, int BN, bool kW8, bool kF8 = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, GemmArgs p) {
@@ -167,9 +172,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_holder;
-    const int KB = p.K / kBK;
+    static_assert(!(kW8 && kF8), "one weight format");
+    constexpr int kKStage = kF8 ? 128 : kBK;  // K elements per stage (128 bytes per row either way)
+    const int KB = p.K / kKStage;
     constexpr uint32_t kTxBytes = SL::kA + (kW8 ? SL::kBq : SL::kBbf);
     constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, BN);
+    constexpr uint32_t kIdescF8 = tc::idesc_e4m3_f32(kBM, BN);
     int issued_round[kStages];  // producer: last round issued on each stage (-1: none)
 #pragma unroll
     for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
@@ -194,15 +202,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     if (p.skip_copy && blockIdx.x == 0 && L == (int)blockIdx.x && kb == 1) continue;
                     tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
-                    tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kBK, a_row0);
+                    tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kKStage, a_row0);
                     if (kW8) {
                         tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
                         if (kDual)
                             tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
                     } else {  // bf16 weights land in the MMA's SWIZZLE_128B tile directly (128 bytes per row)
-                        tc::tma_load_2d(sBbf(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
+                        tc::tma_load_2d(sBbf(s), &tmB0, &full_tma[s], kb * kKStage, w_row0);
                         if (kDual)
-                            tc::tma_load_2d(sBbf(s) + (BN / 2) * 128, &tmB1, &full_tma[s], kb * kBK, w_row0);
+                            tc::tma_load_2d(sBbf(s) + (BN / 2) * 128, &tmB1, &full_tma[s], kb * kKStage, w_row0);
                     }
                     issued_round[s] = r;
                 }
@@ -234,8 +242,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     const uint64_t adesc = tc::sw128_kmajor_desc(tc::smem_u32(sA(s)));
                     const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sBbf(s)));
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes per 16-element K step = +2 in the address field
-                        tc::mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+                    for (int kk = 0; kk < 4; ++kk) {  // +32 bytes per K step (16 bf16 or 32 fp8) = +2 in the address field
+                        if (kF8)
+                            tc::mma_f8_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdescF8, (kb | kk) != 0);
+                        else
+                            tc::mma_bf16_ss(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, kIdesc, (kb | kk) != 0);
+                    }
                     tc::mma_commit(&empty[s]);
                     ++mma_issued;
                 }
@@ -300,7 +312,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tile_coord(hdr, p, L, t);
             const int64_t gr = (int64_t)hdr->seg_start[t.e] + t.m_tile * kBM + row;
             const uint32_t tbase = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
-            if (kDual) {
+            if constexpr (kDual && kF8) {
+                // FP8: scales of the weight rows and of the token's activations; bf16 h in natural k
+                // order (quantized per row by the next kernel)
+                const int j0 = t.n_tile * (BN / 2);
+                const float* s1 = p.sa + (int64_t)t.e * p.N + j0;
+                const float* s3 = p.sb + (int64_t)t.e * p.N + j0;
+                const int32_t a = p.perm[gr];
+                const float as = a >= 0 ? p.a_scale[a / kTopK] : 0.0f;
+                uint4* hrow = reinterpret_cast<uint4*>(p.h_out + gr * p.N + j0);
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    uint32_t a1[32], a3[32];
+                    tc::tmem_ld32(tbase + c, a1);
+                    tc::tmem_ld32(tbase + BN / 2 + c, a3);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int k = 0; k < 8; k += 2) {
+                            const float g0 = __uint_as_float(a1[i + k]) * as * __ldg(s1 + c + i + k);
+                            const float u0 = __uint_as_float(a3[i + k]) * as * __ldg(s3 + c + i + k);
+                            const float g1 = __uint_as_float(a1[i + k + 1]) * as * __ldg(s1 + c + i + k + 1);
+                            const float u1 = __uint_as_float(a3[i + k + 1]) * as * __ldg(s3 + c + i + k + 1);
+                            pk[k / 2] = (uint32_t)f32_to_bf16_bits(silu(g0) * u0) |
+                                        ((uint32_t)f32_to_bf16_bits(silu(g1) * u1) << 16);
+                        }
+                        hrow[(c + i) / 8] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    }
+                }
+            } else if (kDual) {
                 const int j0 = t.n_tile * (BN / 2);
                 const float* s1 = p.sa + (int64_t)t.e * p.N + j0;
                 const float* s3 = p.sb + (int64_t)t.e * p.N + j0;
@@ -338,7 +380,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             } else {
                 const int i0 = t.n_tile * BN;
                 const int32_t a = p.perm[gr];
-                const float wt = a >= 0 ? p.wts[a] : 0.0f;
+                // FP8: the routing weight times the row's activation (h) scale
+                const float wt = a >= 0 ? p.wts[a] * (kF8 ? p.a_scale[gr] : 1.0f) : 0.0f;
                 const float* s2 = p.sa + (int64_t)t.e * p.N + i0;
                 if (p.y_out) {
                     // dense MLP: one assignment per token, its output rounded to bf16 here
@@ -352,9 +395,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                             uint32_t packed[16];
 #pragma unroll
                             for (int i = 0; i < 32; i += 2) {
-                                const float o0 = wt * ((kW8 ? __ldg(s2 + c + i) : 1.0f) * __uint_as_float(v[i]));
+                                const float o0 = wt * ((kW8 || kF8 ? __ldg(s2 + c + i) : 1.0f) * __uint_as_float(v[i]));
                                 const float o1 =
-                                    wt * ((kW8 ? __ldg(s2 + c + i + 1) : 1.0f) * __uint_as_float(v[i + 1]));
+                                    wt * ((kW8 || kF8 ? __ldg(s2 + c + i + 1) : 1.0f) * __uint_as_float(v[i + 1]));
                                 packed[i / 2] =
                                     (uint32_t)f32_to_bf16_bits(o0) | ((uint32_t)f32_to_bf16_bits(o1) << 16);
                             }
@@ -377,10 +420,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
                                 float4 o;
-                                o.x = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
-                                o.y = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
-                                o.z = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
-                                o.w = wt * ((kW8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
+                                o.x = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
+                                o.y = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
+                                o.z = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
+                                o.w = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
                                 dst[k] = o;
                             }
                         }
@@ -460,12 +503,12 @@ int band_for(int K) {
     return b < 1 ? 1 : (b > 16 ? 16 : b);
 }
 
-template <bool kDual, int BN, bool kW8>
+template <bool kDual, int BN, bool kW8, bool kF8 = false>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const GemmArgs& p,
                           int64_t m_tiles_cap, cudaStream_t st) {
     using SL = StageLayout<BN, kW8>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN, kW8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SL::kSmem);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN, kW8, kF8>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (fewer when there are fewer tile slots)
     static int sms_cache[64] = {0};
@@ -476,8 +519,8 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
     }
     int64_t grid = m_tiles_cap * p.n_tiles;
     if (grid > sms) grid = sms;
-    return launch_pdl(gemm_tc_kernel<kDual, BN, kW8>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta, tb0,
-                      tb1, p);
+    return launch_pdl(gemm_tc_kernel<kDual, BN, kW8, kF8>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta,
+                      tb0, tb1, p);
 }
 
 }  // namespace
@@ -556,6 +599,43 @@ cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_
                0};
     if (BN == 256) return launch_gemm_t<false, 256, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
+}
+
+// The FP8 layer's GEMMs: E4M3 activations x8_perm [rows_cap][d] (per-token scales sx, indexed by
+// assignment / K) and weights Q1, Q3 [E][F][d] (scales S1, S3); h = SwiGLU in bf16.
+cudaError_t launch_gemm13_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* x8_perm, const float* sx,
+                             const uint8_t* Q1, const float* S1, const uint8_t* Q3, const float* S3, uint16_t* h,
+                             int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st) {
+    CUtensorMap ta, tb0, tb1;
+    if (!make_map(&ta, x8_perm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows_cap, d, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * F, d, 128, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr,          perm,          S1,          S3,
+               nullptr,      h,             nullptr,     (int)d,
+               (int)F,       (int)(F / 128), band_for((int)d), kMaxPolls,
+               0,            nullptr,       sx};
+    return launch_gemm_t<true, 256, false, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
+}
+
+// out_slot[a] = p_a * sh_r * S2 . (h8_r . Q2^T): E4M3 h8 [rows_cap][F] with per-row scales sh.
+cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h8, const float* sh, const uint8_t* Q2,
+                            const float* S2, const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F,
+                            cudaStream_t st) {
+    const int BN = (d % 256 == 0) ? 256 : 128;
+    CUtensorMap ta, tb0;
+    if (!make_map(&ta, h8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, rows_cap, F, kBM, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)kExperts * d, F, BN, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    GemmArgs p{hdr,         perm,         S2,          nullptr,
+               wts,         nullptr,      out_slot,    (int)F,
+               (int)d,      (int)(d / BN), band_for((int)F), kMaxPolls,
+               0,           nullptr,      sh};
+    if (BN == 256) return launch_gemm_t<false, 256, false, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    return launch_gemm_t<false, 128, false, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
 
 }  // namespace jmoe

@@ -97,6 +97,21 @@ def test_mlp_workspace_and_argument_errors(lib):
     assert mlp(lib, wsb=4096) == 3
 
 
+def test_fp8_workspace_and_argument_errors(lib):
+    assert jm.jamba_moe_workspace_size_fp8(32, 4096, 14336) > 0
+    assert jm.jamba_moe_workspace_size_fp8(8, 4000, 14336) == 0
+    p = [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
+    f = lib.jamba_moe_forward_fp8
+    assert f(None, *p[1:], 8, 256, 512, 16, 2, FAKE, None, None, FAKE, 1 << 40, None, 0) == 1
+    assert f(*p, 8, 256, 512, 8, 2, FAKE, None, None, FAKE, 1 << 40, None, 0) == 2
+    assert f(*p, 8, 256, 512, 16, 2, FAKE + 4, None, None, FAKE, 1 << 40, None, 0) == 7
+    assert f(*p, 8, 256, 512, 16, 2, FAKE, None, None, FAKE, 1024, None, 0) == 3
+    assert f(*p, 8, 256, 512, 16, 2, FAKE, None, None, FAKE, 1 << 40, None, 9) == 2
+    q = lib.jamba_moe_quantize_fp8
+    assert q(None, 1, 4, 16, FAKE, FAKE, None) == 1
+    assert q(FAKE, 1, 4, 10, FAKE, FAKE, None) == 2
+
+
 def test_quantize_argument_errors(lib):
     q = lib.jamba_moe_quantize
     assert q(None, 1, 4, 16, FAKE, FAKE, None) == 1
