@@ -99,7 +99,8 @@ def algorithmic(kind, wl, T, touched, rows_padded, wbytes=1):
 
 
 def kernel_source_hash(kind):
-    files = {"gemv13": ["gemv.cu"], "gemv2": ["gemv.cu"], "gemm13": ["gemm_tc.cu"], "gemm2": ["gemm_tc.cu"],
+    files = {"gemv13": ["gemv.cu"], "gemv2": ["gemv.cu"], "gemm13": ["gemm_tc.cu", "tc.cuh"],
+             "gemm2": ["gemm_tc.cu", "tc.cuh"],
              "quantize": ["quantize.cu"], "router": ["router.cu"], "combine": ["combine.cu"],
              "permute": ["permute.cu"], "gather": ["permute.cu"]}.get(kind, [])
     h = hashlib.sha256()
