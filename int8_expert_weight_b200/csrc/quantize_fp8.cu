@@ -5,12 +5,11 @@
 // infinities, subnormals m * 2^-9).  Used for the weights (per output channel, load time), for the
 // activations x (per token) and for the SwiGLU intermediate h (per permuted row); all bf16 rows.
 //
-// Fast path: the hardware conversion of the fp32 product v * (1/scale) proposes a code c; c is the
-// correctly rounded code whenever the exact residual |v| - |c| * scale lies strictly inside half
-// the spacing of the E4M3 grid on its side of c (see e4m3_check).  Anything else (a tie, or a
-// quotient the fp32 product put on the wrong side of a midpoint) is redone exactly: the fp64
-// quotient (exact enough that no false tie can appear) rounded to the E4M3 grid by power-of-two
-// scaling and rint.
+// Fast path: the hardware conversion of the fp32 product v * (1/scale), whenever that product is
+// provably on the same side of every E4M3 rounding boundary as the exact quotient (see e4m3_safe).
+// Near a boundary (a tie, a near tie, the E4M3 subnormal range) that code is at most one step off
+// and an exact fp32 residual settles it (e4m3_fix); scales below 2^-100 take the fp64 quotient,
+// rounded to the E4M3 grid by power-of-two scaling and rint.
 #include "common.cuh"
 
 namespace jmoe {
@@ -48,35 +47,61 @@ __device__ __noinline__ uint32_t e4m3_exact(float v, float s) {
     return sign | (uint32_t)(((eb + 7) << 3) | ((int)n - 8));
 }
 
-// Is code c (proposed for v / s) the correctly rounded, not tied, one?  v is a bf16 value and s a
-// normal fp32 scale.  The residual d = |v| - |c| s is exact as one fp32 fma: |c| has 4 significant
-// bits and s 24, so |c| s and |v| (8 bits) are multiples of a common quantum q, and whenever
-// |d| < (grid step) * s, |d| / q < 2^24.  Half a grid step times s is exact too (a power of two
-// times s), so the comparisons decide exactly.
-__device__ __forceinline__ bool e4m3_check(float v, float s, uint32_t c) {
-    const uint32_t mc = c & 0x7Fu;
-    if (mc == 0x7Fu) return false;
+// t = v * (1/s) in fp32 is within 2 ulps of the exact quotient q = v / s (two roundings of 2^-24
+// relative each).  E4M3 keeps 3 fraction bits, so in the normal E4M3 range [2^-6, 448) the rounding
+// boundaries of a binade are where the 20 fraction bits below those 3 read 0x80000; if t's bits are
+// more than 3 ulps away from that pattern, no boundary lies between t and q and the hardware rounding
+// of t is the rounding of q.  |t| >= 448 saturates either way; zero is exact; the E4M3 subnormal
+// range and everything else near a boundary go to the exact path.
+__device__ __forceinline__ bool e4m3_safe(float t) {
+    const uint32_t a = __float_as_uint(t) & 0x7FFFFFFFu;
+    if (a >= 0x43E00000u) return true;   // |t| >= 448
+    if (a < 0x3C800000u) return a == 0;  // |t| < 2^-6
+    const int32_t dist = (int32_t)(a & 0xFFFFFu) - 0x80000;
+    return dist > 3 || dist < -3;
+}
+
+// The correctly rounded code of v / s, given a code c at most one step away from it (v a bf16
+// value, s >= 2^-100).  The residual d = |v| - |c| s is exact as one fp32 fma: |c| has 4
+// significant bits and s 24, so |c| s and |v| (8 bits) are multiples of a common quantum q, and
+// |d| < (grid step) * s gives |d| / q < 2^24; half a grid step times s is exact too.  d against
+// half the step on its side decides between c and that neighbour; equality is a tie, to the even
+// code.
+__device__ __noinline__ uint32_t e4m3_fix(float v, float s, uint32_t c) {
+    const uint32_t sign = c & 0x80u, mc = c & 0x7Fu;
     const float d = fmaf(-e4m3_to_f32(mc), s, fabsf(v));
     const uint32_t E = mc >> 3;
-    // half the grid step above c: 2^(max(E,1) - 11); below: half of that at the first code of a
-    // binade (E >= 2), the same otherwise
-    const float half_above = __uint_as_float((127u + (E > 0 ? E : 1u) - 11u) << 23);
+    const float half_above = __uint_as_float((127u + (E > 0 ? E : 1u) - 11u) << 23);  // 2^(max(E,1) - 11)
     const float half_below = ((mc & 7u) == 0 && E >= 2) ? 0.5f * half_above : half_above;
-    if (d >= 0.0f) return mc == 0x7Eu || d < half_above * s;
-    return mc != 0 && -d < half_below * s;
+    uint32_t r = mc;
+    if (d > 0.0f && mc != 0x7Eu) {  // above c (at 448: saturated)
+        const float thr = half_above * s;
+        if (d > thr || (d == thr && (mc & 1u))) r = mc + 1;
+    } else if (d < 0.0f) {
+        const float thr = half_below * s;
+        if (-d > thr || (-d == thr && (mc & 1u))) r = mc - 1;
+    }
+    return sign | r;
 }
 
 // Codes of 8 values (one chunk) as two words, byte i = code of value i.
 __device__ __forceinline__ uint2 fp8_chunk(const float (&v)[8], float s, float inv_s) {
     uint32_t w[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = cvt_e4m3x2(v[2 * i] * inv_s, v[2 * i + 1] * inv_s);
-    bool ok = s >= 0x1p-100f;  // far from fp32's subnormal range, where the products above are exact
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ok &= e4m3_check(v[i], s, (w[i >> 1] >> (8 * (i & 1))) & 0xFFu);
-    if (!ok) {
+    if (s < 0x1p-100f) {  // scales this small: the exact quotient for every value
 #pragma unroll
         for (int i = 0; i < 4; ++i) w[i] = e4m3_exact(v[2 * i], s) | (e4m3_exact(v[2 * i + 1], s) << 8);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float t0 = v[2 * i] * inv_s, t1 = v[2 * i + 1] * inv_s;
+            w[i] = cvt_e4m3x2(t0, t1);
+            const bool ok0 = e4m3_safe(t0), ok1 = e4m3_safe(t1);
+            if (!(ok0 && ok1)) {  // near a rounding boundary: settle it with the exact residual
+                const uint32_t c0 = ok0 ? (w[i] & 0xFFu) : e4m3_fix(v[2 * i], s, w[i] & 0xFFu);
+                const uint32_t c1 = ok1 ? (w[i] >> 8) : e4m3_fix(v[2 * i + 1], s, w[i] >> 8);
+                w[i] = c0 | (c1 << 8);
+            }
+        }
     }
     return make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
 }
