@@ -6,8 +6,11 @@ tensors, passes their device pointers and the current CUDA stream, and turns a n
 into a ``JmoeError``.  PyTorch provides device memory and streams; there is no CPU path.
 
 Functions keep the C names: ``jamba_moe_quantize``, ``jamba_moe_workspace_size``,
-``jamba_moe_forward``, ``jamba_moe_read_device_status``, ``jamba_moe_status_string``,
-``jamba_moe_timing_start``, ``jamba_moe_timing_collect``.
+``jamba_moe_forward`` (the ExpertsInt8 MoE layer), ``jamba_moe_forward_bf16w`` (unquantized bf16
+weights), ``jamba_moe_quantize_fp8`` / ``jamba_moe_workspace_size_fp8`` / ``jamba_moe_forward_fp8``
+(the FP8 comparator layer), ``jamba_mlp_workspace_size`` / ``jamba_mlp_forward`` (the dense
+ExpertsInt8 MLP), ``jamba_moe_forward_noalloc``, ``jamba_moe_read_device_status``,
+``jamba_moe_status_string``, ``jamba_moe_timing_start``, ``jamba_moe_timing_collect``.
 """
 import ctypes
 import os
