@@ -28,7 +28,10 @@
  *     aborts, throws or prints.
  *   - Calls are asynchronous: results are ready when `stream` reaches the point of the call.
  *   - Supported shapes: n_experts == 16, top_k == 2, d and ffn multiples of 128 with
- *     128 <= d, ffn <= 32768, 1 <= T <= 1048576.  Anything else returns JMOE_ERR_SHAPE.
+ *     128 <= d, ffn <= 32768, 0 <= T <= 1048576.  Anything else returns JMOE_ERR_SHAPE.
+ *   - T = 0 (no token) is valid for every forward call but jamba_moe_forward_noalloc: it returns
+ *     JMOE_OK at once, after the size checks, without touching any pointer (they may be NULL) and
+ *     without launching anything.
  */
 #ifndef JMOE_H
 #define JMOE_H
@@ -192,7 +195,7 @@ size_t jamba_mlp_workspace_size(int64_t T, int64_t d, int64_t ffn);
  * It runs the kernels of jamba_moe_forward as a layer of one expert that every token takes with
  * weight 1 (no router, no combine: the down-projection writes y in bf16 directly).  Numerics as
  * in jamba_moe_forward: exact int8 -> bf16, fp32 accumulation, scales on the accumulators, h in
- * bf16; deterministic.  Sizes: 1 <= T <= 1<<20, d and ffn multiples of 128 in [128, 32768];
+ * bf16; deterministic.  Sizes: 0 <= T <= 1<<20, d and ffn multiples of 128 in [128, 32768];
  * x, y, Q1, Q3, Q2 16-byte aligned, scales 4-byte aligned.  Errors as in jamba_moe_forward.
  */
 int jamba_mlp_forward(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,

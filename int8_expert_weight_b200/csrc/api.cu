@@ -75,7 +75,7 @@ struct Layout {
 
 bool shape_ok(int64_t T, int64_t d, int64_t F, int E, int K) {
     if (E != kExperts || K != kTopK) return false;
-    if (T < 1 || T > kMaxT) return false;
+    if (T < 0 || T > kMaxT) return false;
     if (d < 128 || d > kMaxDim || d % 128 != 0) return false;
     if (F < 128 || F > kMaxDim || F % 128 != 0) return false;
     return true;
@@ -177,10 +177,11 @@ int forward_impl(const uint16_t* x, const float* router_W, const float* router_b
                  const float* S1, const void* W3, const float* S3, const void* W2, const float* S2, bool w8,
                  int64_t T, int64_t d, int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids,
                  float* topk_w, void* workspace, size_t workspace_bytes, void* stream, int path) {
-    if (!x || !router_W || !W1 || !W3 || !W2 || !y || !workspace) return JMOE_ERR_NULL;
-    if (w8 && (!S1 || !S3 || !S2)) return JMOE_ERR_NULL;
     if (!shape_ok(T, d, ffn, n_experts, top_k)) return JMOE_ERR_SHAPE;
     if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    if (T == 0) return JMOE_OK;  // no token: nothing to read or write
+    if (!x || !router_W || !W1 || !W3 || !W2 || !y || !workspace) return JMOE_ERR_NULL;
+    if (w8 && (!S1 || !S3 || !S2)) return JMOE_ERR_NULL;
     const void* ptrs16[] = {x, W1, W3, W2, y, router_W};
     for (const void* p : ptrs16)
         if (!aligned16(p)) return JMOE_ERR_ALIGN;
@@ -292,9 +293,10 @@ Layout make_layout_mlp(int64_t T, int64_t d, int64_t F) {
 int mlp_impl(const uint16_t* x, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
              const int8_t* Q2, const float* S2, int64_t T, int64_t d, int64_t ffn, uint16_t* y, void* workspace,
              size_t workspace_bytes, void* stream, int path) {
-    if (!x || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
     if (!shape_ok(T, d, ffn, kExperts, kTopK)) return JMOE_ERR_SHAPE;
     if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    if (T == 0) return JMOE_OK;
+    if (!x || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
     const void* ptrs16[] = {x, Q1, Q3, Q2, y};
     for (const void* p : ptrs16)
         if (!aligned16(p)) return JMOE_ERR_ALIGN;
@@ -384,9 +386,10 @@ int forward_f8(const uint16_t* x, const float* router_W, const float* router_bia
                const uint8_t* Q3, const float* S3, const uint8_t* Q2, const float* S2, int64_t T, int64_t d,
                int64_t ffn, int n_experts, int top_k, uint16_t* y, int32_t* topk_ids, float* topk_w, void* workspace,
                size_t workspace_bytes, void* stream, int path) {
-    if (!x || !router_W || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
     if (!shape_ok(T, d, ffn, n_experts, top_k)) return JMOE_ERR_SHAPE;
     if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    if (T == 0) return JMOE_OK;
+    if (!x || !router_W || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !y || !workspace) return JMOE_ERR_NULL;
     const void* ptrs16[] = {x, Q1, Q3, Q2, y, router_W};
     for (const void* p : ptrs16)
         if (!aligned16(p)) return JMOE_ERR_ALIGN;

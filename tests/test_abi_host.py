@@ -37,7 +37,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_workspace_size(lib):
     assert jm.jamba_moe_workspace_size(32, 4096, 14336) > 32 * 2 * 4096 * 4
-    assert jm.jamba_moe_workspace_size(0, 4096, 14336) == 0
+    assert jm.jamba_moe_workspace_size(0, 4096, 14336) > 0      # no token: valid, nothing to do
+    assert jm.jamba_moe_workspace_size(-1, 4096, 14336) == 0
     assert jm.jamba_moe_workspace_size(8, 4000, 14336) == 0      # d not a multiple of 128
     assert jm.jamba_moe_workspace_size(8, 4096, 14336, 8, 2) == 0  # only 16 experts
     assert jm.jamba_moe_workspace_size(8, 4096, 14336, 16, 1) == 0  # only top-2
@@ -68,7 +69,10 @@ def test_forward_argument_errors(lib):
     assert fwd(lib, K=1) == 2
     assert fwd(lib, d=200) == 2
     assert fwd(lib, F=100) == 2
-    assert fwd(lib, T=0) == 2
+    assert fwd(lib, T=-1) == 2
+    assert fwd(lib, T=0) == 0                      # no token: nothing launched
+    assert fwd(lib, T=0, x=None, y=None, ws=None, wsb=0) == 0  # and no pointer read
+    assert fwd(lib, T=0, d=200) == 2               # sizes are still checked
     assert fwd(lib, path=7) == 2
     assert fwd(lib, x=FAKE + 8) == 7
     assert fwd(lib, ws=FAKE + 16) == 3
@@ -83,12 +87,13 @@ def test_mlp_workspace_and_argument_errors(lib):
     a = jm.jamba_mlp_workspace_size(32, 4096, 14336)
     assert a > 128 * 14336 * 2 and a % 256 == 0
     assert a < jm.jamba_moe_workspace_size(32, 4096, 14336)
-    assert jm.jamba_mlp_workspace_size(0, 4096, 14336) == 0
+    assert jm.jamba_mlp_workspace_size(-1, 4096, 14336) == 0
     assert jm.jamba_mlp_workspace_size(8, 4096, 14300) == 0
     assert mlp(lib, x=None) == 1
     assert mlp(lib, s=None) == 1
     assert mlp(lib, ws=None) == 1
-    assert mlp(lib, T=0) == 2
+    assert mlp(lib, T=-1) == 2
+    assert mlp(lib, T=0, x=None, y=None, ws=None, s=None) == 0
     assert mlp(lib, d=200) == 2
     assert mlp(lib, path=5) == 2
     assert mlp(lib, y=FAKE + 2) == 7

@@ -137,3 +137,37 @@ def test_large_decode_all_paths():
         y, ids, w = L.forward(path=path)
         ref = L.oracle_forward(tokens=toks)
         assert_y_close(y[toks], ref["y"], f"large decode path {path}")
+
+
+@pytest.mark.parametrize("path", PATHS)
+def test_two_experts_take_every_token(path):
+    """A router bias that sends every token to experts 5 and 9: fourteen experts get no token (their
+    weights are never read) and two get all 300, in segments of three 128-row tiles each."""
+    wl = dataclasses.replace(workload("tiny"), T=300, bias={5: 30.0, 9: 30.0})
+    L = Layer(wl)
+    check_layer(L, path)
+    assert set(np.unique(L.forward(path)[1]).tolist()) == {5, 9}
+
+
+def test_no_token_is_a_no_op():
+    """T = 0 on every forward entry point: no error, empty outputs."""
+    d, F, E = 256, 512, 16
+    dev = "cuda"
+    x = torch.empty((0, d), dtype=torch.bfloat16, device=dev)
+    wr = torch.zeros((E, d), dtype=torch.float32, device=dev)
+    q13 = torch.zeros((E, F, d), dtype=torch.int8, device=dev)
+    q2 = torch.zeros((E, d, F), dtype=torch.int8, device=dev)
+    s13 = torch.ones((E, F), dtype=torch.float32, device=dev)
+    s2 = torch.ones((E, d), dtype=torch.float32, device=dev)
+    for path in (jm.PATH_AUTO, jm.PATH_GEMV, jm.PATH_GEMM):
+        y, ids, w = jm.jamba_moe_forward(x, wr, None, q13, s13, q13, s13, q2, s2, path=path)
+        assert y.shape == (0, d) and ids.shape == (0, 2) and w.shape == (0, 2)
+        y, _, _ = jm.jamba_moe_forward_bf16w(x, wr, None, q13.to(torch.bfloat16), q13.to(torch.bfloat16),
+                                            q2.to(torch.bfloat16), path=path)
+        assert y.shape == (0, d)
+        y, _, _ = jm.jamba_moe_forward_fp8(x, wr, None, q13.view(torch.uint8), s13, q13.view(torch.uint8), s13,
+                                          q2.view(torch.uint8), s2, path=path)
+        assert y.shape == (0, d)
+        y = jm.jamba_mlp_forward(x, q13[0], s13[0], q13[0], s13[0], q2[0], s2[0], path=path)
+        assert y.shape == (0, d)
+    torch.cuda.synchronize()
