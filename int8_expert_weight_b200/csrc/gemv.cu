@@ -1,7 +1,7 @@
 // Decode path of the expert FFN: few tokens per expert, so the work is bound by streaming the
-// int8 weights from HBM (Jamba rebuttal page, reply on MoE and Mamba layer interaction: MLP/MoE
-// layers are I/O bound; Jamba-1.5 paper, §3.1: the weights cross HBM -> SRAM as int8, half the
-// bytes of BF16, and are turned into BF16 right before the math).
+// int8 weights from HBM (Jamba rebuttal page, reply on MoE and Mamba layer interaction: these
+// layers are limited by memory traffic, not arithmetic; Jamba-1.5 paper, §3.1: the weights cross
+// HBM -> SRAM as int8, half the bytes of BF16, and are turned into BF16 right before the math).
 //
 //   gemv13: h[r][j]      = bf16( SiLU(S1[j] * (x_r . Q1[j])) * (S3[j] * (x_r . Q3[j])) )
 //   gemv2:  out[a][i]    = p_a * S2[i] * (h_r . Q2[i])        (a = the assignment of permuted row r)

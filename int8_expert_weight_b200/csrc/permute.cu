@@ -1,6 +1,7 @@
 // Expert histogram, padded prefix sum and stable token permutation (the batching of tokens per
 // expert that lets each expert run as one GEMM; Jamba rebuttal page, reply on MoE and Mamba layer
-// interaction: the two experts of a token are computed independently, so batching and fusing pay).
+// interaction: a token's two experts are independent pieces of work, which is what lets them be
+// grouped by expert).
 //
 // One CTA of 1024 threads:
 //   1. histogram of the T*K routing assignments (shared-memory integer atomics: exact),
