@@ -1,0 +1,58 @@
+"""Host-side pieces of bench.py that the JSON line depends on: the algorithmic work per launch that
+divides into the roofline, and the source key that decides whether a stored ncu traffic figure
+still belongs to the kernel being timed (a stale figure is reported as null)."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+
+def test_algorithmic_work_of_the_decode_workload():
+    wl = synth.WORKLOADS["v01_decode"]
+    d, F, T = wl.d, wl.F, wl.T
+    kind, b13 = bench.algorithmic("gemv13", wl, T, touched=16, rows_padded=2048)
+    assert kind == "bytes"
+    # every touched expert's W1 and W3 once (int8 codes + fp32 row scales), x rows in, h rows out
+    assert b13 == 16 * (2 * F * d + 2 * F * 4) + 2 * T * d * 2 + 2 * T * F * 2
+    kind, b2 = bench.algorithmic("gemv2", wl, T, touched=16, rows_padded=2048)
+    assert kind == "bytes" and b2 == 16 * (d * F + d * 4) + 2 * T * F * 2 + 2 * T * d * 4 + 2 * T * 8
+    # bf16 weights: twice the weight bytes, no scales
+    _, b13w = bench.algorithmic("gemv13", wl, T, 16, 2048, wbytes=2)
+    assert b13w == 16 * (2 * F * d * 2) + 2 * T * d * 2 + 2 * T * F * 2
+    # fewer touched experts: fewer weight bytes
+    assert bench.algorithmic("gemv13", wl, T, 5, 2048)[1] < b13
+
+
+def test_algorithmic_flops_of_the_prefill_workload():
+    wl = synth.WORKLOADS["v01_prefill"]
+    kind, f13 = bench.algorithmic("gemm13", wl, wl.T, 16, 0)
+    assert kind == "flops" and f13 == 2.0 * (2 * wl.T) * wl.d * (2 * wl.F)
+    kind, f2 = bench.algorithmic("gemm2", wl, wl.T, 16, 0)
+    assert kind == "flops" and f2 == 2.0 * (2 * wl.T) * wl.F * wl.d
+
+
+def test_algorithmic_work_of_the_dense_mlp():
+    wl = synth.MLP_WORKLOADS["mlp_v01_decode"]
+    d, F, T = wl.d, wl.F, wl.T
+    # one weight set, every token once; the down-projection writes y in bf16
+    assert bench.algorithmic("gemv2", wl, T, 1, 128)[1] == d * F + d * 4 + T * F * 2 + T * d * 2
+    assert bench.algorithmic("gemm13", synth.MLP_WORKLOADS["mlp_v01_prefill"], 8192, 1, 0)[1] == \
+        2.0 * 8192 * d * 2 * F
+
+
+def test_source_key_ignores_comments_only(tmp_path, monkeypatch):
+    csrc = tmp_path / "int8_expert_weight_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "common.cuh").write_text("// header\nint a;\n")
+    (csrc / "gemv.cu").write_text("/* notes */\nint f() { return 1; }  // one\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    k0 = bench.kernel_source_hash("gemv13")
+    (csrc / "gemv.cu").write_text("/* other notes,\n   two lines */\nint f() { return 1; }  // uno\n")
+    assert bench.kernel_source_hash("gemv13") == k0
+    (csrc / "gemv.cu").write_text("int f() { return 2; }\n")
+    assert bench.kernel_source_hash("gemv13") != k0
+
