@@ -21,8 +21,9 @@
  *     The library allocates no device memory, never synchronises the stream (except where
  *     stated) and launches its kernels only on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).
- *   - Tensors are dense, row-major, with the last dimension contiguous.  Device pointers must
- *     be 16-byte aligned.
+ *   - Tensors are dense, row-major, with the last dimension contiguous.  Activation, weight and
+ *     output pointers must be 16-byte aligned; scale, bias and routing-output pointers 4-byte
+ *     aligned; workspaces 256-byte aligned (JMOE_ERR_ALIGN / JMOE_ERR_WORKSPACE otherwise).
  *   - Calls return a jmoe_status.  Argument errors are detected on the host before anything is
  *     launched and leave all buffers untouched.  Launch failures return JMOE_ERR_CUDA.  No call
  *     aborts, throws or prints.
