@@ -19,6 +19,12 @@
 //
 // Tiles are ordered expert by expert; inside an expert, bands of M tiles keep their activations
 // resident in L2 while every N tile of the weights streams past once per band.
+//
+// The same kernel serves three weight formats (template flags): int8 codes (kW8, the layer above),
+// unquantized bf16 weights (TMA straight into the MMA's tile, 4 stages, converters idle), and the
+// FP8 comparator (kF8: E4M3 activations and weights, both by TMA, 128 K elements per stage,
+// kind::f8f6f4 MMAs, per-row activation scales in the epilogue, bf16 h).  The W2 epilogue can also
+// write y in bf16 directly (the dense MLP, one assignment per token) instead of fp32 slots.
 #include <cuda.h>
 
 #include "common.cuh"
