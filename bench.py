@@ -104,14 +104,15 @@ def kernel_source_hash(kind):
              "gemm2": ["gemm_tc.cu", "tc.cuh"],
              "quantize": ["quantize.cu"], "router": ["router.cu"], "combine": ["combine.cu"],
              "permute": ["permute.cu"], "gather": ["permute.cu"]}.get(kind, [])
-    # the code only: comments are stripped, so an edit of a comment keeps a capture valid
+    # the code only: comments are stripped and whitespace collapsed, so an edit of a comment keeps a
+    # capture valid
     h = hashlib.sha256()
     for f in files + ["common.cuh"]:
         p = os.path.join(ROOT, "int8_expert_weight_b200", "csrc", f)
         if os.path.exists(p):
             src = re.sub(r"/\*.*?\*/", "", open(p).read(), flags=re.S)
             src = re.sub(r"//[^\n]*", "", src)
-            h.update(src.encode())
+            h.update(" ".join(src.split()).encode())  # layout-insensitive: whitespace runs count as one
     return h.hexdigest()[:16]
 
 

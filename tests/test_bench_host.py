@@ -53,6 +53,9 @@ def test_source_key_ignores_comments_only(tmp_path, monkeypatch):
     k0 = bench.kernel_source_hash("gemv13")
     (csrc / "gemv.cu").write_text("/* other notes,\n   two lines */\nint f() { return 1; }  // uno\n")
     assert bench.kernel_source_hash("gemv13") == k0
+    # a comment block removed with its lines, re-indented code: still the same key
+    (csrc / "gemv.cu").write_text("\n\n\nint  f()\n{ return 1; }\n")
+    assert bench.kernel_source_hash("gemv13") == k0
     (csrc / "gemv.cu").write_text("int f() { return 2; }\n")
     assert bench.kernel_source_hash("gemv13") != k0
 
