@@ -151,13 +151,14 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
     return d;
 }
 
-// Instruction descriptor for kind::f16: bf16 A and B, fp32 D, both K-major, shape M x N.
-// kind::f8f6f4 with both operands E4M3 (format code 0), fp32 accumulation, K-major A and B.
+// Instruction descriptor for kind::f8f6f4 with both operands E4M3 (format code 0), fp32
+// accumulation, K-major A and B, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
     return (1u << 4)                        // D format: f32
            | ((uint32_t)(N >> 3) << 17)     // N / 8
            | ((uint32_t)(M >> 4) << 24);    // M / 16
 }
+// Instruction descriptor for kind::f16: bf16 A and B, fp32 D, both K-major, shape M x N.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4)                        // D format: f32
            | (1u << 7)                      // A format: bf16
