@@ -93,8 +93,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     return lib
 
 
-def _stream_ptr(stream: Optional[torch.cuda.Stream]) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device: Optional[torch.device] = None) -> int:
+    """The stream to launch on: the given one, else the current stream of `device`."""
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    if device is not None and s.device != device:
+        raise ValueError(f"stream belongs to {s.device}, the tensors to {device}")
     return s.cuda_stream
 
 
@@ -109,6 +112,17 @@ def _check(t: torch.Tensor, name: str, dtype: torch.dtype, shape=None):
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _one_device(ref: torch.Tensor, **tensors) -> torch.device:
+    """The device of `ref`, after checking that every other tensor of the call is on it too.  The
+    call then runs with that device current, on its stream: the library launches on the current
+    device."""
+    for name, t in tensors.items():
+        if t is not None and t.device != ref.device:
+            raise ValueError(f"{name} is on {t.device}, the call's first tensor on {ref.device}: "
+                             "every tensor of a call must be on one device")
+    return ref.device
 
 
 def jamba_moe_status_string(status: int) -> str:
@@ -136,7 +150,10 @@ def jamba_moe_quantize(W: torch.Tensor, stream: Optional[torch.cuda.Stream] = No
         Q, S = out
         _check(Q, "Q", torch.int8, W.shape)
         _check(S, "S", torch.float32, W.shape[:-1])
-    st = lib.jamba_moe_quantize(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(), _stream_ptr(stream))
+    dev = _one_device(W, Q=Q, S=S)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_quantize(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(),
+                                    _stream_ptr(stream, dev))
     if st != 0:
         raise JmoeError(st, "jamba_moe_quantize")
     return Q, S
@@ -190,10 +207,13 @@ def jamba_moe_forward(x: torch.Tensor, router_W: torch.Tensor, router_bias: Opti
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     _check(workspace, "workspace", torch.uint8)
     p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
-    st = lib.jamba_moe_forward_path(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
-                                    S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
-                                    T, d, ffn, E, TOP_K, y.data_ptr(), p(topk_ids), p(topk_w),
-                                    workspace.data_ptr(), workspace.numel(), _stream_ptr(stream), int(path))
+    dev = _one_device(x, router_W=router_W, router_bias=router_bias, Q1=Q1, S1=S1, Q3=Q3, S3=S3, Q2=Q2, S2=S2, y=y,
+                      topk_ids=topk_ids, topk_w=topk_w, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_forward_path(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
+                                        S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
+                                        T, d, ffn, E, TOP_K, y.data_ptr(), p(topk_ids), p(topk_w),
+                                        workspace.data_ptr(), workspace.numel(), _stream_ptr(stream, dev), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward")
     return y, topk_ids, topk_w
@@ -216,7 +236,10 @@ def jamba_moe_quantize_fp8(W: torch.Tensor, stream: Optional[torch.cuda.Stream] 
         Q, S = out
         _check(Q, "Q", torch.uint8, W.shape)
         _check(S, "S", torch.float32, W.shape[:-1])
-    st = lib.jamba_moe_quantize_fp8(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(), _stream_ptr(stream))
+    dev = _one_device(W, Q=Q, S=S)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_quantize_fp8(W.data_ptr(), n_mats, rows, cols, Q.data_ptr(), S.data_ptr(),
+                                        _stream_ptr(stream, dev))
     if st != 0:
         raise JmoeError(st, "jamba_moe_quantize_fp8")
     return Q, S
@@ -266,10 +289,13 @@ def jamba_moe_forward_fp8(x: torch.Tensor, router_W: torch.Tensor, router_bias: 
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     _check(workspace, "workspace", torch.uint8)
     p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
-    st = lib.jamba_moe_forward_fp8(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(), S1.data_ptr(),
-                                   Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(), T, d, ffn, E, TOP_K,
-                                   y.data_ptr(), p(topk_ids), p(topk_w), workspace.data_ptr(), workspace.numel(),
-                                   _stream_ptr(stream), int(path))
+    dev = _one_device(x, router_W=router_W, router_bias=router_bias, Q1=Q1, S1=S1, Q3=Q3, S3=S3, Q2=Q2, S2=S2, y=y,
+                      topk_ids=topk_ids, topk_w=topk_w, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_forward_fp8(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
+                                       S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(), T, d,
+                                       ffn, E, TOP_K, y.data_ptr(), p(topk_ids), p(topk_w), workspace.data_ptr(),
+                                       workspace.numel(), _stream_ptr(stream, dev), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward_fp8")
     return y, topk_ids, topk_w
@@ -307,9 +333,11 @@ def jamba_mlp_forward(x: torch.Tensor, Q1: torch.Tensor, S1: torch.Tensor, Q3: t
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     _check(workspace, "workspace", torch.uint8)
-    st = lib.jamba_mlp_forward_path(x.data_ptr(), Q1.data_ptr(), S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(),
-                                    Q2.data_ptr(), S2.data_ptr(), T, d, ffn, y.data_ptr(), workspace.data_ptr(),
-                                    workspace.numel(), _stream_ptr(stream), int(path))
+    dev = _one_device(x, Q1=Q1, S1=S1, Q3=Q3, S3=S3, Q2=Q2, S2=S2, y=y, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_mlp_forward_path(x.data_ptr(), Q1.data_ptr(), S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(),
+                                        Q2.data_ptr(), S2.data_ptr(), T, d, ffn, y.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel(), _stream_ptr(stream, dev), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_mlp_forward")
     return y
@@ -345,10 +373,13 @@ def jamba_moe_forward_bf16w(x: torch.Tensor, router_W: torch.Tensor, router_bias
         workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
     _check(workspace, "workspace", torch.uint8)
     p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
-    st = lib.jamba_moe_forward_bf16w(x.data_ptr(), router_W.data_ptr(), p(router_bias), W1.data_ptr(), W3.data_ptr(),
-                                     W2.data_ptr(), T, d, ffn, E, TOP_K, y.data_ptr(), topk_ids.data_ptr(),
-                                     topk_w.data_ptr(), workspace.data_ptr(), workspace.numel(), _stream_ptr(stream),
-                                     int(path))
+    dev = _one_device(x, router_W=router_W, router_bias=router_bias, W1=W1, W3=W3, W2=W2, y=y, topk_ids=topk_ids,
+                      topk_w=topk_w, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_forward_bf16w(x.data_ptr(), router_W.data_ptr(), p(router_bias), W1.data_ptr(),
+                                         W3.data_ptr(), W2.data_ptr(), T, d, ffn, E, TOP_K, y.data_ptr(),
+                                         topk_ids.data_ptr(), topk_w.data_ptr(), workspace.data_ptr(),
+                                         workspace.numel(), _stream_ptr(stream, dev), int(path))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward_bf16w")
     return y, topk_ids, topk_w
@@ -370,10 +401,13 @@ def jamba_moe_forward_noalloc(x: torch.Tensor, router_W: torch.Tensor, router_bi
                      (topk_ids, "topk_ids", torch.int32), (topk_w, "topk_w", torch.float32)):
         _check(t, n, dt)
     p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
-    st = lib.jamba_moe_forward_noalloc(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
-                                       S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
-                                       T, d, ffn, E, TOP_K, y.data_ptr(), topk_ids.data_ptr(), topk_w.data_ptr(),
-                                       _stream_ptr(stream))
+    dev = _one_device(x, router_W=router_W, router_bias=router_bias, Q1=Q1, S1=S1, Q3=Q3, S3=S3, Q2=Q2, S2=S2, y=y,
+                      topk_ids=topk_ids, topk_w=topk_w)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_forward_noalloc(x.data_ptr(), router_W.data_ptr(), p(router_bias), Q1.data_ptr(),
+                                           S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(), S2.data_ptr(),
+                                           T, d, ffn, E, TOP_K, y.data_ptr(), topk_ids.data_ptr(), topk_w.data_ptr(),
+                                           _stream_ptr(stream, dev))
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward_noalloc")
     return y, topk_ids, topk_w
@@ -382,7 +416,9 @@ def jamba_moe_forward_noalloc(x: torch.Tensor, router_W: torch.Tensor, router_bi
 def jamba_moe_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
     """Synchronise the stream and return the device status word of the last forward on workspace."""
     _check(workspace, "workspace", torch.uint8)
-    return int(load_library().jamba_moe_read_device_status(workspace.data_ptr(), _stream_ptr(stream)))
+    with torch.cuda.device(workspace.device):
+        return int(load_library().jamba_moe_read_device_status(workspace.data_ptr(),
+                                                               _stream_ptr(stream, workspace.device)))
 
 
 def jamba_moe_debug_skip_copy(on: bool) -> None:
