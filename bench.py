@@ -485,7 +485,7 @@ def run_ours(args):
             "metric": METRIC_MLP if mlp else METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
             "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
                            weights=("int8 codes + fp32 per-output-channel scales" if int8w else
                                     "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
