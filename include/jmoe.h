@@ -2,9 +2,9 @@
  * jmoe.h — C ABI of the ExpertsInt8 mixture-of-experts layer for NVIDIA B200 (sm_100a).
  *
  * The layer (Jamba-1.5: Hybrid Transformer-Mamba Models at Scale, "Model Architecture":
- * n = 16 experts, the top K = 2 chosen at each token; §3.1 "ExpertsInt8": expert weights are
- * quantized to INT8, stored in INT8 and turned back into BF16 inside the fused MoE kernel,
- * right before the matrix math) computes, for every token x_t (a row of d bf16 values):
+ * n = 16 experts, two of them serving every token; §3.1 "ExpertsInt8": expert weights are kept
+ * as 8-bit integer codes and converted into BF16 inside the fused MoE kernel just before the
+ * matrix math) computes, for every token x_t (a row of d bf16 values):
  *
  *     z_e   = sum_i x_ti * Wr[e][i] (+ b_e)                  router logits, fp32
  *     p     = softmax(z)                                      over all 16 experts
@@ -141,7 +141,7 @@ int jamba_moe_forward_bf16w(const uint16_t* x, const float* router_W, const floa
 
 /*
  * FP8 comparator layer.  The Jamba-1.5 paper (§3.1) compares ExpertsInt8 with FP8 serving (on H100,
- * ExpertsInt8 matches FP8's latency; FP8 needs FP8 hardware and, unlike ExpertsInt8, does not keep
+ * the two run with equal latency; FP8 needs FP8 hardware and, unlike ExpertsInt8, does not keep
  * BF16 activations) without defining the FP8 scheme.  This library's reading: both GEMM operands
  * are OCP FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
  * finite 448, subnormals m * 2^-9); weights carry one fp32 scale per output channel, the

@@ -15,7 +15,7 @@
  *     which decides every tie exactly for a bf16 w and an fp32 scale), and an
  *     all-zero row gets scale 1 and q = 0.
  *   - oracle_route: the MoE router (Jamba-1.5 paper, "Model Architecture":
- *     n = 16 experts, the top K = 2 selected at each token).  Readings: logits
+ *     n = 16 experts, two of them serving every token).  Readings: logits
  *     z_e = sum_i x_i * Wr[e][i] (+ bias_e), softmax over all E experts,
  *     the K largest logits in descending order (equal logits: lower expert
  *     index first), weights = the softmax probabilities of the chosen experts,
@@ -25,8 +25,8 @@
  *   - oracle_moe_forward: y_t = sum_k w_tk * E_{e_tk}(x_t) with SwiGLU experts
  *     E_e(x) = W2_e (SiLU(W1_e x) * (W3_e x)) (GLU variants, Shazeer 2020,
  *     cited by the Jamba paper), where each weight is the dequantized value
- *     q * scale formed exactly in fp64 (Jamba-1.5 paper, §3.1: weights are
- *     dequantized back before the computation).  No intermediate rounding:
+ *     q * scale formed exactly in fp64 (Jamba-1.5 paper, §3.1: the int8 weights
+ *     become BF16 values again for the arithmetic).  No intermediate rounding:
  *     the result is fp64.
  *   - oracle_quantize_rows_fp8, oracle_moe_forward_fp8: the FP8 (E4M3) layer the
  *     Jamba-1.5 paper compares ExpertsInt8 with (§3.1), per-channel weight scales and
