@@ -3,7 +3,7 @@
  *
  * The layer (Jamba-1.5: Hybrid Transformer-Mamba Models at Scale, "Model Architecture":
  * n = 16 experts, two of them serving every token; §3.1 "ExpertsInt8": expert weights are kept
- * as 8-bit integer codes and converted into BF16 inside the fused MoE kernel just before the
+ * as 8-bit integer codes and converted into BF16 inside the expert GEMM kernel just before the
  * matrix math) computes, for every token x_t (a row of d bf16 values):
  *
  *     z_e   = sum_i x_ti * Wr[e][i] (+ b_e)                  router logits, fp32
@@ -182,7 +182,7 @@ size_t jamba_mlp_workspace_size(int64_t T, int64_t d, int64_t ffn);
 /*
  * jamba_mlp_forward — the dense MLP of the layers without MoE, on ExpertsInt8 weights (Jamba-1.5
  * paper, §3.1: the MLP weights are quantized and dequantized like the experts'; "Model
- * Architecture": MoE takes the place of the MLP only every e = 2 layers):
+ * Architecture": one layer in e = 2 has an MoE block, the other an MLP):
  *
  *     y_t = bf16( S2 * (Q2 . h_t) ),  h_t = bf16( SiLU(S1 * (Q1 . x_t)) * (S3 * (Q3 . x_t)) )
  *

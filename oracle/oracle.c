@@ -400,8 +400,8 @@ int oracle_moe_forward_bf16w(const uint16_t* x, int64_t T, int64_t d, int64_t F,
 /* ------------------------------------------------------------- dense MLP */
 
 /* The MLP of a layer without MoE, with ExpertsInt8 weights (Jamba-1.5 paper, §3.1 "ExpertsInt8":
- * the MLP weights are quantized like the experts'; "Model Architecture": MoE replaces the single
- * MLP only every e = 2 layers).  The MLP is the same SwiGLU block as one expert,
+ * the MLP weights are quantized like the experts'; "Model Architecture": one layer in e = 2 has
+ * an MoE block, the other an MLP).  The MLP is the same SwiGLU block as one expert,
  *   y_t = W2 (SiLU(W1 x_t) * (W3 x_t)),  w = q * scale formed exactly in fp64,
  * taken by every token with weight 1: no router, no softmax, no sum over experts. */
 static void mlp_range(void* p, int64_t b, int64_t e) {

@@ -130,8 +130,8 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 
-# The dense MLP of the layers without MoE (Jamba-1.5 paper, "Model Architecture": MoE replaces the
-# MLP every e = 2 layers; §3.1: ExpertsInt8 quantizes the MLP weights too), with the expert's shape.
+# The dense MLP of the layers without MoE (Jamba-1.5 paper, "Model Architecture": one layer in e = 2 has an
+# MoE block, the other an MLP; §3.1: ExpertsInt8 quantizes the MLP weights too), with the expert's shape.
 MLP_WORKLOADS: Dict[str, Workload] = {
     w.name: w
     for w in [
