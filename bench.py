@@ -221,7 +221,8 @@ def oracle_forward(wl, setup, tokens, threads):
 
 
 def oracle_rate(wl, setup, budget_s, max_tokens=None):
-    """Tokens/s of the oracle forward on a bounded sample (tokens spread over the batch)."""
+    """Tokens/s of the oracle forward on a bounded sample (tokens spread over the batch), with the
+    sampled tokens and the oracle's result on them."""
     import oracle
     threads = oracle.default_threads()
     t0 = time.perf_counter()
@@ -232,10 +233,30 @@ def oracle_rate(wl, setup, budget_s, max_tokens=None):
         n = min(n, max_tokens)
     toks = np.linspace(0, wl.T - 1, n).round().astype(np.int64)
     t0 = time.perf_counter()
-    oracle_forward(wl, setup, toks, threads)
+    ref = oracle_forward(wl, setup, toks, threads)
     dt = time.perf_counter() - t0
     used = min(threads, n)
-    return n / dt, used, n, dt
+    return n / dt, used, n, dt, toks, ref
+
+
+def parity_stats(y_bits, ids, ref):
+    """The layer's parity measures on sampled tokens: y_bits bf16 bits [n][d] and ids int32 [n][K]
+    (None for the dense MLP) from the GPU, ref the oracle's result on the same tokens.  The bench
+    batch is not filtered for near-tied router logits, so a token may legitimately take another
+    pair of experts; such tokens are counted and left out of the y measures."""
+    y = synth.bf16_bits_to_f32(np.asarray(y_bits, np.uint16)).astype(np.float64)
+    r = np.asarray(ref["y"], np.float64)
+    same = np.ones(len(r), bool)
+    out = {"tokens": int(len(r))}
+    if ids is not None and "ids" in ref:
+        same = (np.sort(np.asarray(ids), 1) == np.sort(ref["ids"], 1)).all(1)
+        out["id_mismatch_tokens"] = int((~same).sum())
+    err = np.abs(y[same] - r[same])
+    den = np.abs(r[same]).sum()
+    out["max_err_rel"] = float((err / (1.0 + np.abs(r[same]))).max()) if err.size else 0.0
+    out["mean_rel_err"] = float(err.sum() / den) if den > 0 else 0.0
+    out["within_tolerance"] = bool(out["max_err_rel"] <= 2e-2 and out["mean_rel_err"] <= 5e-3)
+    return out
 
 
 def run_reference(args):
@@ -473,12 +494,17 @@ def run_ours(args):
         per_kernel[k] = {"launches": n, "avg_us": kms / n * 1e3,
                          ("GB/s" if uk == "bytes" else "TFLOP/s"): a / (1e9 if uk == "bytes" else 1e12)}
 
-    cpu = None
+    cpu = parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and int8w:
         setup = oracle_setup(wl, seed_x)
-        rate, cores, n, dt = oracle_rate(wl, setup, args.cpu_budget_s)
+        rate, cores, n, dt, toks, ref = oracle_rate(wl, setup, args.cpu_budget_s)
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} of {wl.T} tokens (evenly spaced) of the same batch, fp64, {dt:.1f} s"}
+        try:  # the last forward's output on the oracle's sample: a record, never a reason to fail the run
+            y_bits = y.view(torch.int16).cpu().numpy().view(np.uint16)[toks]
+            parity = parity_stats(y_bits, None if mlp else ids.cpu().numpy()[toks], ref)
+        except Exception as ex:  # noqa: BLE001
+            parity = {"error": repr(ex)[:200]}
 
     if rank == 0:
         out = {
@@ -491,7 +517,7 @@ def run_ours(args):
                                     "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
                                     "per-row scales (FP8 comparator)" if fp8 else
                                     "bf16 (unquantized comparator)")),
-            "roofline": roofline, "cpu_baseline": cpu,
+            "roofline": roofline, "cpu_baseline": cpu, "parity_on_sample": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 2},
             "gpu_launches": int(sum(n for _, n in kernels.values())),

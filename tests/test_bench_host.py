@@ -4,6 +4,8 @@ still belongs to the kernel being timed (a stale figure is reported as null)."""
 import os
 import sys
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
 
@@ -84,3 +86,27 @@ def test_reference_arm_prints_one_contract_line():
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_parity_on_sample_measures():
+    """parity_stats, which puts the sampled GPU-vs-oracle comparison into the bench line: the
+    oracle's own output rounded to bf16 is within tolerance, a 10 % error is not, and a token whose
+    expert pair differs is counted and left out of the y measures."""
+    wl = synth.WORKLOADS["tiny"]
+    setup = bench.oracle_setup(wl, wl.seed)
+    toks = np.arange(0, wl.T, 5)
+    ref = bench.oracle_forward(wl, setup, toks, 1)
+    y_bits = synth.f32_to_bf16_bits(ref["y"].astype(np.float32))
+    ok = bench.parity_stats(y_bits, ref["ids"], ref)
+    assert ok["tokens"] == len(toks) and ok["id_mismatch_tokens"] == 0 and ok["within_tolerance"]
+    assert 0 < ok["max_err_rel"] < 1e-2 and ok["mean_rel_err"] < 5e-3
+    bad = bench.parity_stats(synth.f32_to_bf16_bits((ref["y"] * 1.1).astype(np.float32)), ref["ids"], ref)
+    assert not bad["within_tolerance"]
+    ids = ref["ids"].copy()
+    ids[3] = (ids[3] + 1) % 16
+    y_off = y_bits.copy()
+    y_off[3] = synth.f32_to_bf16_bits(np.full(wl.d, 1e3, np.float32))  # that token's y is then unrelated
+    mism = bench.parity_stats(y_off, ids, ref)
+    assert mism["id_mismatch_tokens"] == 1 and mism["within_tolerance"]
+    mlp = bench.parity_stats(y_bits, None, {"y": ref["y"]})
+    assert "id_mismatch_tokens" not in mlp and mlp["within_tolerance"]
