@@ -28,6 +28,9 @@
  *     launched and leave all buffers untouched.  Launch failures return JMOE_ERR_CUDA.  No call
  *     aborts, throws or prints.
  *   - Calls are asynchronous: results are ready when `stream` reaches the point of the call.
+ *   - Host threads: the quantize, workspace-size and forward calls may be made from several
+ *     threads at once (each with its own workspace and outputs); the timing calls, the test hooks
+ *     and jamba_moe_forward_noalloc (one shared scratch array) may not.
  *   - Supported shapes: n_experts == 16, top_k == 2, d and ffn multiples of 128 with
  *     128 <= d, ffn <= 32768, 0 <= T <= 1048576.  Anything else returns JMOE_ERR_SHAPE.
  *   - T = 0 (no token) is valid for every forward call but jamba_moe_forward_noalloc: it returns

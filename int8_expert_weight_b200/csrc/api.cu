@@ -1,5 +1,6 @@
 // C ABI of the ExpertsInt8 MoE layer: argument checks, workspace layout, kernel sequencing and
 // the optional per-launch event timing.  Declared in include/jmoe.h.
+#include <atomic>
 #include <vector>
 
 #include "common.cuh"
@@ -108,16 +109,18 @@ Layout make_layout(int64_t T, int64_t d, int64_t F) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// SM count of the current device, looked up once per device (relaxed atomics: several host
+// threads may race to fill an entry, all with the same value).
 int num_sms_current() {
-    static int cache[64] = {0};
+    static std::atomic<int> cache[64];  // zero-initialised (static storage)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (cache[dev] == 0) {
-        int n = 0;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // ---------------------------------------------------------------- launch timing

@@ -27,6 +27,8 @@
 // write y in bf16 directly (the dense MLP, one assignment per token) instead of fp32 slots.
 #include <cuda.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -473,17 +475,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// Looked up once; the initialisation of a function-local static is thread-safe.
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void* f = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(f);
-    }
+            return reinterpret_cast<EncodeTiledFn>(f);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -517,11 +518,13 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (fewer when there are fewer tile slots)
-    static int sms_cache[64] = {0};
+    static std::atomic<int> sms_cache[64];  // per device; zero-initialised (static storage)
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64) {
-        if (!sms_cache[dev]) cudaDeviceGetAttribute(&sms_cache[dev], cudaDevAttrMultiProcessorCount, dev);
-        if (sms_cache[dev] > 0) sms = sms_cache[dev];
+        int n = sms_cache[dev].load(std::memory_order_relaxed);
+        if (n <= 0 && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+            sms_cache[dev].store(n, std::memory_order_relaxed);
+        if (n > 0) sms = n;
     }
     int64_t grid = m_tiles_cap * p.n_tiles;
     if (grid > sms) grid = sms;
