@@ -131,12 +131,14 @@ def test_large_prefill_sampled():
 
 @pytest.mark.slow
 def test_large_decode_all_paths():
+    """The 1.5-Large decode shape (9.7 GB of int8 experts): every token, both expert paths."""
     L = Layer(workload("large_decode"))
-    toks = np.arange(0, 64, 4)
+    ref = L.oracle_forward()
+    _, _, z = oracle.route(L.x_bits, L.wr, L.bias, want_logits=True)
     for path in (jm.PATH_AUTO, jm.PATH_GEMM):
         y, ids, w = L.forward(path=path)
-        ref = L.oracle_forward(tokens=toks)
-        assert_y_close(y[toks], ref["y"], f"large decode path {path}")
+        assert_routing(ids, w, ref["ids"], ref["w"], z)
+        assert_y_close(y, ref["y"], f"large decode path {path}")
 
 
 @pytest.mark.parametrize("path", PATHS)
