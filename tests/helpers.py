@@ -82,3 +82,47 @@ def assert_routing(ids_gpu: np.ndarray, w_gpu: np.ndarray, ids_ref: np.ndarray, 
     same = ids_gpu == ids_ref
     w_ref_matched = np.where(same, w_ref, w_ref[:, ::-1])
     assert np.max(np.abs(w_gpu.astype(np.float64) - w_ref_matched)) <= W_ABS
+
+
+def expert_segments(ids: np.ndarray, n_experts: int = 16):
+    """Per expert, the assignment indices a = t*K + k routed to it in the order of its permuted
+    segment (ascending a: the permutation is stable, so token order)."""
+    flat = np.asarray(ids).reshape(-1)
+    return [np.nonzero(flat == e)[0] for e in range(n_experts)]
+
+
+def tile_covering_tokens(ids: np.ndarray, n_min: int = 512, tile: int = 128, seed: int = 0) -> np.ndarray:
+    """Tokens to compare with the oracle on a large batch: one row drawn (seeded) from every
+    `tile`-row M tile of every expert's permuted segment, the first and last row of every segment,
+    then evenly strided tokens until at least `n_min` distinct tokens (or all T) are taken."""
+    ids = np.asarray(ids)
+    T, K = ids.shape
+    rng = np.random.default_rng(seed)
+    toks = set()
+    for seg in expert_segments(ids):
+        if seg.size == 0:
+            continue
+        toks.update([int(seg[0] // K), int(seg[-1] // K)])
+        for m0 in range(0, seg.size, tile):
+            rows = seg[m0:m0 + tile]
+            toks.add(int(rows[rng.integers(rows.size)] // K))
+    n = min(n_min, T)
+    extra = n_min
+    while len(toks) < n:
+        toks.update(np.linspace(0, T - 1, extra).round().astype(int).tolist())
+        extra *= 2
+    return np.array(sorted(toks), dtype=np.int64)
+
+
+def uncovered_tiles(ids: np.ndarray, tokens: np.ndarray, tile: int = 128):
+    """(expert, M tile) pairs of the permuted order none of whose rows belongs to `tokens`."""
+    ids = np.asarray(ids)
+    K = ids.shape[1]
+    chosen = np.zeros(ids.shape[0], bool)
+    chosen[np.asarray(tokens)] = True
+    missing = []
+    for e, seg in enumerate(expert_segments(ids)):
+        for m, m0 in enumerate(range(0, seg.size, tile)):
+            if not chosen[seg[m0:m0 + tile] // K].any():
+                missing.append((e, m))
+    return missing

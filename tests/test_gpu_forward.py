@@ -13,7 +13,8 @@ pytestmark = pytest.mark.gpu
 
 import int8_expert_weight_b200 as jm  # noqa: E402
 from gpu_layer import Layer  # noqa: E402
-from helpers import assert_routing, assert_y_close, workload  # noqa: E402
+from helpers import (assert_routing, assert_y_close, tile_covering_tokens, uncovered_tiles,  # noqa: E402
+                     workload)
 import oracle  # noqa: E402
 
 PATHS = [pytest.param(jm.PATH_GEMV, id="gemv"), pytest.param(jm.PATH_GEMM, id="gemm")]
@@ -89,24 +90,15 @@ def test_v01_decode_gemm_path(v01_decode):
     check_layer(v01_decode, jm.PATH_GEMM)
 
 
-def sample_tokens(ids_ref: np.ndarray, n_strided: int) -> np.ndarray:
-    """Evenly strided tokens plus, for every expert, the first and last token routed to it (the first
-    and last rows of its permuted segment, since the permutation keeps token order)."""
-    T = ids_ref.shape[0]
-    toks = set(np.linspace(0, T - 1, n_strided).round().astype(int).tolist())
-    for e in range(16):
-        hit = np.nonzero((ids_ref == e).any(1))[0]
-        if hit.size:
-            toks.update([int(hit[0]), int(hit[-1]), int(hit[hit.size // 2])])
-    return np.array(sorted(toks), dtype=np.int64)
-
-
-def check_sampled(L: Layer, path, n_strided):
+def check_sampled(L: Layer, path):
+    """Routing on every token; y on tokens that cover every (expert, 128-row M tile) of the permuted
+    order (at least 512), computed by the oracle one token at a time."""
     assert all(v == 0 for v in L.quant_mismatch.values()), L.quant_mismatch
     y, ids, w = L.forward(path=path)
     ids_o, w_o, z = oracle.route(L.x_bits, L.wr, L.bias, want_logits=True)
     assert_routing(ids, w, ids_o, w_o, z)  # every token
-    toks = sample_tokens(ids_o, n_strided)
+    toks = tile_covering_tokens(ids_o)
+    assert toks.size >= 512 and uncovered_tiles(ids_o, toks) == []
     ref = L.oracle_forward(tokens=toks)
     return assert_y_close(y[toks], ref["y"], f"y on {toks.size} sampled tokens")
 
@@ -117,16 +109,16 @@ def v01_prefill():
 
 
 def test_v01_prefill_sampled(v01_prefill):
-    check_sampled(v01_prefill, jm.PATH_AUTO, 256)
+    check_sampled(v01_prefill, jm.PATH_AUTO)
 
 
 def test_skewed_sampled():
-    check_sampled(Layer(workload("skewed")), jm.PATH_AUTO, 256)
+    check_sampled(Layer(workload("skewed")), jm.PATH_AUTO)
 
 
 @pytest.mark.slow
 def test_large_prefill_sampled():
-    check_sampled(Layer(workload("large_prefill")), jm.PATH_AUTO, 96)
+    check_sampled(Layer(workload("large_prefill")), jm.PATH_AUTO)
 
 
 @pytest.mark.slow

@@ -19,7 +19,8 @@ import int8_expert_weight_b200 as jm  # noqa: E402
 import oracle  # noqa: E402
 import synth  # noqa: E402
 from gpu_layer import bf16_to_dev, dev_to_bf16_bits  # noqa: E402
-from helpers import assert_routing, assert_y_close, gap_inputs, workload  # noqa: E402
+from helpers import (assert_routing, assert_y_close, gap_inputs, tile_covering_tokens,  # noqa: E402
+                     uncovered_tiles, workload)
 from oracle_pins import E4M3_VALUES, bf16_bits  # noqa: E402
 
 PATHS = [pytest.param(jm.PATH_GEMV, id="gemv"), pytest.param(jm.PATH_GEMM, id="gemm")]
@@ -123,5 +124,7 @@ def test_fp8_v01_decode_all_tokens():
 
 def test_fp8_v01_prefill_sampled():
     L = F8Layer(workload("v01_prefill"))
-    toks = np.linspace(0, L.wl.T - 1, 128).round().astype(np.int64)
+    ids_o, _, _ = oracle.route(L.x_bits, L.wr, L.bias, want_logits=True)
+    toks = tile_covering_tokens(ids_o)
+    assert toks.size >= 512 and uncovered_tiles(ids_o, toks) == []
     check(L, jm.PATH_AUTO, toks)

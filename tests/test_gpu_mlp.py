@@ -14,7 +14,7 @@ import int8_expert_weight_b200 as jm  # noqa: E402
 import oracle  # noqa: E402
 import synth  # noqa: E402
 from gpu_layer import bf16_to_dev, dev_to_bf16_bits  # noqa: E402
-from helpers import assert_y_close  # noqa: E402
+from helpers import assert_y_close, tile_covering_tokens, uncovered_tiles  # noqa: E402
 
 PATHS = [pytest.param(jm.PATH_GEMV, id="gemv"), pytest.param(jm.PATH_GEMM, id="gemm")]
 
@@ -107,5 +107,7 @@ def test_mlp_v01_decode_all_tokens():
 def test_mlp_v01_prefill_sampled():
     L = Mlp(mlp_workload("mlp_v01_prefill"))
     y = L.forward(jm.PATH_AUTO)
-    toks = np.unique(np.concatenate([np.linspace(0, L.wl.T - 1, 96).round(), [127, 128, 8191]]).astype(np.int64))
+    one_expert = np.zeros((L.wl.T, 1), np.int32)  # the MLP's rows are its tokens, in order
+    toks = tile_covering_tokens(one_expert)
+    assert toks.size >= 512 and uncovered_tiles(one_expert, toks) == []
     assert_y_close(y[toks], L.ref(tokens=toks))
