@@ -31,7 +31,7 @@ import synth  # noqa: E402
 METRIC = "MoE-layer tokens/sec (int8 experts) at 1 B200; % of HBM / BF16 roofline"
 METRIC_MLP = "dense-MLP tokens/sec (ExpertsInt8 weights) at 1 B200; % of HBM / BF16 roofline"
 UNIT = "tokens/s"
-DEFAULT_WORKLOAD = "v01_decode"
+DEFAULT_WORKLOAD = "skewed"  # the largest single-GPU configuration: T=65536, d=4096, ffn=14336
 
 
 def parse():
@@ -286,13 +286,22 @@ def run_reference(args):
         "metric": METRIC if wl.layer == "moe" else METRIC_MLP, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": workload_config(wl, "oracle"),
+        "config": run_config(wl, args, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, n), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(out), flush=True)
     return 0
+
+
+def run_config(wl, args, world):
+    """The `config` object of both arms' JSON lines (the same keys and values for the same run)."""
+    fp8, int8w = args.weights == "fp8", args.weights == "int8"
+    return dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
+                weights=("int8 codes + fp32 per-output-channel scales" if int8w else
+                         "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
+                         "per-row scales (FP8 comparator)" if fp8 else "bf16 (unquantized comparator)"))
 
 
 def workload_config(wl, path):
@@ -413,7 +422,7 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    status = jm.jamba_moe_read_device_status(ws)
+    status = {"warmup": jm.jamba_moe_read_device_status(ws)}  # JMOE_OK = 0 after each pass
     ids_np = np.zeros((T, 1), np.int32) if mlp else ids.cpu().numpy()
     touched = int(np.unique(ids_np).size)
     counts = np.bincount(ids_np.reshape(-1), minlength=E)
@@ -444,6 +453,7 @@ def run_ours(args):
     with ClockSampler(local_rank) as clk:
         ms_plain, _ = timed_pass(False)
         ms_events, kernels = timed_pass(True)
+    status["timed"] = jm.jamba_moe_read_device_status(ws)
     ms = max_over_ranks(ms_plain, dev)
     ms_events = max_over_ranks(ms_events, dev)
     value = aggregate_tokens_per_s(world, T, args.steps, ms)
@@ -468,6 +478,7 @@ def run_ours(args):
         step_e2e()
     ev1.record(stream)
     torch.cuda.synchronize()
+    status["e2e"] = jm.jamba_moe_read_device_status(ws)
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     e2e_value = aggregate_tokens_per_s(world, T, args.steps, e2e_ms)
 
@@ -479,14 +490,23 @@ def run_ours(args):
     if unit_kind == "bytes":
         achieved, peak, unit, bound = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
     else:
-        # FP8 MMAs: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
-        achieved, peak, unit, bound = (work / avg_s / 1e12, peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0),
+        # the burst bf16 peak (each kernel is timed alone by its own events); FP8 MMAs: the measured
+        # bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        achieved, peak, unit, bound = (work / avg_s / 1e12, peaks["bf16_tflops"] * (2.0 if fp8 else 1.0),
                                        "TFLOP/s", "tensor")
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
                 "traffic": ncu_traffic(dom, wl.name) if args.weights == "int8" else None, "kernel": dom,
                 "algorithmic_per_launch": work,
-                "peak_source": peaks["source"] + (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 and bound == "tensor"
-                                                  else "")}
+                "peak_source": peaks["source"] + (" burst" if bound == "tensor" else "") +
+                               (" bf16 x 2 (nominal fp8/bf16 ratio)" if fp8 and bound == "tensor" else "")}
+    if bound == "tensor":
+        sus = peaks["bf16_tflops_sustained"] * (2.0 if fp8 else 1.0)
+        roofline["peak_sustained"] = sus
+        roofline["frac_of_sustained"] = achieved / sus
+    clocks = clk.summary()
+    if clocks.get("sm_mhz"):
+        # the same rate per SM clock: comparable across runs that ran at different clocks
+        roofline["achieved_per_sm_mhz"] = achieved / clocks["sm_mhz"]
     per_kernel = {}
     for k, (kms, n) in sorted(kernels.items(), key=lambda kv: -kv[1][0]):
         uk, wk = algorithmic(k, wl, T, touched, rows_padded, wbytes)
@@ -512,17 +532,13 @@ def run_ours(args):
             "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3" if fp8 else "bf16", "data": "synthetic",
-            "config": dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
-                           weights=("int8 codes + fp32 per-output-channel scales" if int8w else
-                                    "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
-                                    "per-row scales (FP8 comparator)" if fp8 else
-                                    "bf16 (unquantized comparator)")),
+            "config": run_config(wl, args, world),
             "roofline": roofline, "cpu_baseline": cpu, "parity_on_sample": parity,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * d * 2,
                     "d2h_bytes_per_step": T * d * 2},
             "gpu_launches": int(sum(n for _, n in kernels.values())),
             "ms_per_step_with_kernel_events": ms_events / args.steps,
-            "clocks": clk.summary(), "kernels": per_kernel, "device_status": status,
+            "clocks": clocks, "kernels": per_kernel, "device_status": status,
             "routing": {"touched_experts": touched, "max_tokens_per_expert": int(counts.max())},
             "quantize": ({"ms": q_ms, "GB/s": q_bytes / (q_ms / 1e3) / 1e9,
                           "frac_of_hbm": q_bytes / (q_ms / 1e3) / 1e9 / peaks["hbm_gbs"]} if q_ms > 0 else None),
