@@ -257,6 +257,13 @@ int jamba_moe_forward_noalloc(const uint16_t* x, const float* router_W, const fl
 size_t jamba_moe_noalloc_scratch_capacity(void);
 /* Scratch bytes jamba_moe_forward_noalloc needs for these sizes (0 = unsupported sizes). */
 size_t jamba_moe_noalloc_scratch_needed(int64_t T, int64_t d, int64_t ffn);
+/*
+ * jamba_moe_noalloc_read_device_status — jamba_moe_read_device_status for the static scratch of
+ * jamba_moe_forward_noalloc on the current device: synchronises `stream`, then returns the status
+ * word its last call left there (JMOE_OK, JMOE_DEV_TIMEOUT or JMOE_DEV_BAD_INDEX); JMOE_ERR_CUDA
+ * if the lookup or the 4-byte copy fails.  Allocates nothing.
+ */
+int jamba_moe_noalloc_read_device_status(void* stream);
 
 /*
  * Kernel timing (for the benchmark's roofline figures).

@@ -82,6 +82,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jamba_moe_noalloc_scratch_capacity.argtypes = []
     lib.jamba_moe_noalloc_scratch_needed.restype = sz
     lib.jamba_moe_noalloc_scratch_needed.argtypes = [i64, i64, i64]
+    lib.jamba_moe_noalloc_read_device_status.restype = c_int
+    lib.jamba_moe_noalloc_read_device_status.argtypes = [vp]
     lib.jamba_moe_forward_bf16w.restype = c_int
     lib.jamba_moe_forward_bf16w.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, c_int, c_int, vp, vp, vp, vp, sz,
                                             vp, c_int]
@@ -411,6 +413,15 @@ def jamba_moe_forward_noalloc(x: torch.Tensor, router_W: torch.Tensor, router_bi
     if st != 0:
         raise JmoeError(st, "jamba_moe_forward_noalloc")
     return y, topk_ids, topk_w
+
+
+def jamba_moe_noalloc_read_device_status(device=None, stream: Optional[torch.cuda.Stream] = None) -> int:
+    """Synchronise the stream and return the device status word that the last
+    jamba_moe_forward_noalloc call on `device` (default: the current device) left in the static
+    scratch."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(load_library().jamba_moe_noalloc_read_device_status(_stream_ptr(stream, dev)))
 
 
 def jamba_moe_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

@@ -9,8 +9,11 @@
 //     library, from load until process exit.
 //   - The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
 //     that device current; make that first call before any stream capture.
-//   - All calls share the array and it keeps the last call's contents.  Each call first clears
-//     the routing header, then every other byte it reads is written earlier in the same call.
+//   - All calls share the array and it keeps the last call's contents.  Every byte a call reads
+//     is written earlier in the same call (the permutation kernel rewrites the routing header,
+//     status word included); the header is also cleared at the start of each call, as a defence.
+//   - jamba_moe_noalloc_read_device_status reads the array's status word (the device-side error
+//     report of the last call on the current device).
 //   - Two calls that may overlap on the GPU (other streams, other host threads) race on the array.
 //   - Sizes whose scratch does not fit return JMOE_ERR_WORKSPACE.
 //   - No cudaMalloc, cudaFree or allocating library routine is called.
@@ -119,7 +122,8 @@ extern "C" int jamba_moe_forward_noalloc(const uint16_t* x, const float* router_
     float* slots = reinterpret_cast<float*>(p);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the header carries counts and the status word from the previous call: start it from zero
+    // defensive: the permutation kernel rewrites every header field the later kernels read, the
+    // status word included, but a header left over from an earlier call is cleared all the same
     if (cudaMemsetAsync(hdr, 0, kHeaderBytes, st) != cudaSuccess) return JMOE_ERR_CUDA;
     if (launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st) != cudaSuccess)
         return JMOE_ERR_CUDA;
@@ -128,4 +132,19 @@ extern "C" int jamba_moe_forward_noalloc(const uint16_t* x, const float* router_
     if (launch_gemv2(hdr, perm, h, Q2, S2, wts, slots, T, d, ffn, st) != cudaSuccess) return JMOE_ERR_CUDA;
     if (launch_combine(slots, T, d, y, st, sms) != cudaSuccess) return JMOE_ERR_CUDA;
     return JMOE_OK;
+}
+
+// The status word of the static scratch on the current device: what the kernels of the last
+// jamba_moe_forward_noalloc call there reported (JMOE_OK, JMOE_DEV_TIMEOUT or JMOE_DEV_BAD_INDEX).
+// Synchronises `stream` first; reads 4 bytes into a host variable, allocates nothing.
+extern "C" int jamba_moe_noalloc_read_device_status(void* stream) {
+    void* base = nullptr;
+    int sms = 0;
+    const int rc = scratch_for_current_device(&base, &sms);
+    if (rc != JMOE_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t status = 0;
+    if (cudaMemcpyAsync(&status, base, sizeof(status), cudaMemcpyDeviceToHost, st) != cudaSuccess) return JMOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return JMOE_ERR_CUDA;
+    return (int)status;
 }

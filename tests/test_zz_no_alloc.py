@@ -14,7 +14,8 @@ pytestmark = pytest.mark.gpu
 
 import int8_expert_weight_b200 as jm  # noqa: E402
 from gpu_layer import Layer, dev_to_bf16_bits  # noqa: E402
-from helpers import assert_y_close, workload  # noqa: E402
+from helpers import assert_routing, assert_y_close, workload  # noqa: E402
+import oracle  # noqa: E402
 
 
 @pytest.fixture(scope="module")
@@ -52,6 +53,26 @@ def test_noalloc_matches_forward_twice(lib, name, over):
         assert np.array_equal(ids.cpu().numpy(), ids_ref)
         assert np.max(np.abs(w.cpu().numpy() - w_ref)) <= 1e-5
         assert_y_close(dev_to_bf16_bits(y), ref, "noalloc y vs jamba_moe_forward")
+
+
+def test_noalloc_against_oracle_and_status(lib):
+    """The allocation-free call checked straight against the fp64 oracle (not only against the
+    workspace call), through the Python wrapper on a side stream, and its device status word read
+    back from the static scratch."""
+    L = Layer(workload("tiny", T=48, d=512, F=768))
+    wl = L.wl
+    ref = L.oracle_forward()
+    side = torch.cuda.Stream()
+    y = torch.empty((wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty((wl.T, 2), dtype=torch.int32, device="cuda")
+    w = torch.empty((wl.T, 2), dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()  # the inputs were written on the default stream
+    jm.jamba_moe_forward_noalloc(L.x, L.wr_dev, L.bias_dev, L.q["w1"], L.s["w1"], L.q["w3"], L.s["w3"], L.q["w2"],
+                                 L.s["w2"], y=y, topk_ids=ids, topk_w=w, stream=side)
+    assert jm.jamba_moe_noalloc_read_device_status(stream=side) == 0
+    _, _, z = oracle.route(L.x_bits, L.wr, L.bias, want_logits=True)
+    assert_routing(ids.cpu().numpy(), w.cpu().numpy(), ref["ids"], ref["w"], z)
+    assert_y_close(dev_to_bf16_bits(y), ref["y"], "noalloc y vs oracle")
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
