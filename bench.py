@@ -46,6 +46,9 @@ def parse():
     ap.add_argument("--weights", default="int8", choices=["int8", "bf16", "fp8"],
                     help="int8: ExpertsInt8 (the method); bf16: the unquantized comparator layer; "
                          "fp8: the FP8 (E4M3 weights and activations) comparator layer")
+    ap.add_argument("--parallel", default="replicas", choices=["replicas", "ep"],
+                    help="replicas: every rank runs the whole layer on its own batch (no collective); "
+                         "ep: experts split over the ranks, rows exchanged by NCCL all-to-all")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     return ap.parse_args()
@@ -298,7 +301,9 @@ def run_reference(args):
 def run_config(wl, args, world):
     """The `config` object of both arms' JSON lines (the same keys and values for the same run)."""
     fp8, int8w = args.weights == "fp8", args.weights == "int8"
-    return dict(workload_config(wl, args.path), parallelism=f"replicas{world}" if world > 1 else "1gpu",
+    par = (f"ep{world}" if getattr(args, "parallel", "replicas") == "ep" else
+           f"replicas{world}" if world > 1 else "1gpu")
+    return dict(workload_config(wl, args.path), parallelism=par,
                 weights=("int8 codes + fp32 per-output-channel scales" if int8w else
                          "E4M3 codes + fp32 per-output-channel scales; E4M3 activations with "
                          "per-row scales (FP8 comparator)" if fp8 else "bf16 (unquantized comparator)"))
@@ -350,13 +355,26 @@ def run_ours(args):
     rank, local_rank, world = dist_env()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    if world > 1:
+    ep = args.parallel == "ep"
+    if world > 1 or ep:
         import datetime
+        if world == 1:  # a one-rank group for the expert-parallel path on a single GPU
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     wl = synth.ALL_WORKLOADS[args.workload]
     mlp = wl.layer == "mlp"
     if mlp and args.weights != "int8":
         raise SystemExit("the dense MLP workloads run with ExpertsInt8 weights only")
+    if ep and (mlp or args.weights != "int8"):
+        raise SystemExit("the expert-parallel path runs the MoE layer with ExpertsInt8 weights")
+    if ep:
+        from int8_expert_weight_b200.ep import CudaSteps, ep_forward, expert_range
+        e_first, e_last = expert_range(rank, world)
+    else:
+        e_first, e_last = 0, wl.E
     T, d, F, E = wl.T, wl.d, wl.F, wl.E
     path = {"auto": jm.PATH_AUTO, "gemv": jm.PATH_GEMV, "gemm": jm.PATH_GEMM}[args.path]
     peaks = load_peaks()
@@ -377,9 +395,9 @@ def run_ours(args):
     jm.jamba_moe_timing_start(3)  # the quantize launches (one per matrix), timed by the library's own events
     for which in ("w1", "w3", "w2"):
         rows, cols = synth.weight_shape(wl, which)
-        Wb[which] = torch.empty((E, rows, cols), dtype=torch.bfloat16, device=dev)
-        for e in range(E):  # drawn expert by expert on the host, to bound host memory
-            Wb[which][e].copy_(to_dev(synth.gen_expert(wl, which, e)))
+        Wb[which] = torch.empty((e_last - e_first, rows, cols), dtype=torch.bfloat16, device=dev)
+        for e in range(e_first, e_last):  # drawn expert by expert on the host, to bound host memory
+            Wb[which][e - e_first].copy_(to_dev(synth.gen_expert(wl, which, e)))
         if int8w:
             Q[which], S[which] = jm.jamba_moe_quantize(Wb[which])
             del Wb[which]
@@ -398,8 +416,16 @@ def run_ours(args):
     tw = torch.empty((T, 2), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    ep_stats = {}
+    ep_steps = CudaSteps(path) if ep else None
+    y_ep = [y]
+
     def forward(xin):
-        if mlp:
+        if ep:
+            y_ep[0], ids_ep, _ = ep_forward(xin, wr, bias, (Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"]),
+                                            steps=ep_steps, stats=ep_stats)
+            ids.copy_(ids_ep)
+        elif mlp:
             jm.jamba_mlp_forward(xin, Q["w1"][0], S["w1"][0], Q["w3"][0], S["w3"][0], Q["w2"][0], S["w2"][0], y=y,
                                  workspace=ws, path=path)
         elif int8w:
@@ -422,10 +448,22 @@ def run_ours(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
-    status = {"warmup": jm.jamba_moe_read_device_status(ws)}  # JMOE_OK = 0 after each pass
-    ids_np = np.zeros((T, 1), np.int32) if mlp else ids.cpu().numpy()
-    touched = int(np.unique(ids_np).size)
-    counts = np.bincount(ids_np.reshape(-1), minlength=E)
+    def read_status():
+        if ep:  # the expert-parallel calls keep their own workspaces: the worse of the two
+            return max(ep_steps.dispatch_status(), ep_steps.experts_status())
+        return jm.jamba_moe_read_device_status(ws)
+
+    status = {"warmup": read_status()}  # JMOE_OK = 0 after each pass
+    T_work = T  # tokens whose assignments this rank's expert kernels process
+    if ep:
+        # this rank's kernels work on the rows it received, one assignment each
+        counts = np.bincount(ep_stats["recv_expert"].cpu().numpy(), minlength=E)
+        touched = int((counts > 0).sum())
+        T_work = sum(ep_stats["recv_counts"]) / wl.K
+    else:
+        ids_np = np.zeros((T, 1), np.int32) if mlp else ids.cpu().numpy()
+        touched = int(np.unique(ids_np).size)
+        counts = np.bincount(ids_np.reshape(-1), minlength=E)
     rows_padded = int(sum((c + 127) // 128 * 128 for c in counts))
 
     # ---- timed region: K forward steps on resident inputs.  A CUDA event recorded between two
@@ -453,7 +491,7 @@ def run_ours(args):
     with ClockSampler(local_rank) as clk:
         ms_plain, _ = timed_pass(False)
         ms_events, kernels = timed_pass(True)
-    status["timed"] = jm.jamba_moe_read_device_status(ws)
+    status["timed"] = read_status()
     ms = max_over_ranks(ms_plain, dev)
     ms_events = max_over_ranks(ms_events, dev)
     value = aggregate_tokens_per_s(world, T, args.steps, ms)
@@ -467,7 +505,7 @@ def run_ours(args):
     def step_e2e():
         x_dev.copy_(x_host, non_blocking=True)
         forward(x_dev)
-        y_host.copy_(y, non_blocking=True)
+        y_host.copy_(y_ep[0] if ep else y, non_blocking=True)
 
     for _ in range(args.warmup):
         step_e2e()
@@ -478,14 +516,14 @@ def run_ours(args):
         step_e2e()
     ev1.record(stream)
     torch.cuda.synchronize()
-    status["e2e"] = jm.jamba_moe_read_device_status(ws)
+    status["e2e"] = read_status()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     e2e_value = aggregate_tokens_per_s(world, T, args.steps, e2e_ms)
 
     # ---- roofline of the dominant kernel
     dom = max(kernels, key=lambda k: kernels[k][0])
     dom_ms, dom_n = kernels[dom]
-    unit_kind, work = algorithmic(dom, wl, T, touched, rows_padded, wbytes)
+    unit_kind, work = algorithmic(dom, wl, T_work, touched, rows_padded, wbytes)
     avg_s = dom_ms / dom_n / 1e3
     if unit_kind == "bytes":
         achieved, peak, unit, bound = work / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
@@ -509,7 +547,7 @@ def run_ours(args):
         roofline["achieved_per_sm_mhz"] = achieved / clocks["sm_mhz"]
     per_kernel = {}
     for k, (kms, n) in sorted(kernels.items(), key=lambda kv: -kv[1][0]):
-        uk, wk = algorithmic(k, wl, T, touched, rows_padded, wbytes)
+        uk, wk = algorithmic(k, wl, T_work, touched, rows_padded, wbytes)
         a = wk / (kms / n / 1e3)
         per_kernel[k] = {"launches": n, "avg_us": kms / n * 1e3,
                          ("GB/s" if uk == "bytes" else "TFLOP/s"): a / (1e9 if uk == "bytes" else 1e12)}
@@ -521,7 +559,7 @@ def run_ours(args):
         cpu = {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
                "sample": f"{n} of {wl.T} tokens (evenly spaced) of the same batch, fp64, {dt:.1f} s"}
         try:  # the last forward's output on the oracle's sample: a record, never a reason to fail the run
-            y_bits = y.view(torch.int16).cpu().numpy().view(np.uint16)[toks]
+            y_bits = (y_ep[0] if ep else y).view(torch.int16).cpu().numpy().view(np.uint16)[toks]
             parity = parity_stats(y_bits, None if mlp else ids.cpu().numpy()[toks], ref)
         except Exception as ex:  # noqa: BLE001
             parity = {"error": repr(ex)[:200]}

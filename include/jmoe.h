@@ -55,7 +55,9 @@ typedef enum {
     JMOE_ERR_CUDA = 4,       /* a CUDA runtime call or kernel launch failed */
     JMOE_DEV_TIMEOUT = 5,    /* a kernel gave up waiting on a pipeline barrier (device status) */
     JMOE_DEV_BAD_INDEX = 6,  /* a kernel saw an out-of-range routing index (device status) */
-    JMOE_ERR_ALIGN = 7       /* a pointer is not 16-byte aligned */
+    JMOE_ERR_ALIGN = 7,      /* a pointer is not 16-byte aligned */
+    JMOE_DEV_BAD_TABLE = 8,  /* debug checks: the routing tables are not a valid permutation (device status) */
+    JMOE_DEV_CANARY = 9      /* debug checks: a workspace guard gap was overwritten (device status) */
 } jmoe_status;
 
 /* Forward-path selection for jamba_moe_forward_path. */
@@ -235,6 +237,31 @@ const char* jamba_moe_status_string(int status);
 int jamba_moe_debug_skip_copy(int on);
 
 /*
+ * jamba_moe_debug_checks — debug checks, off by default.  While `on` is non-zero, every MoE
+ * forward call (jamba_moe_forward, _path, _bf16w, _fp8) also launches: at its start, a kernel that
+ * fills the guard gaps the workspace layout leaves after each of its regions with a canary pattern;
+ * after the permutation, a kernel that checks the routing tables (counts sum to T*K, every
+ * expert's segment is its count rounded up to 128 rows, each permuted row holds -1 or an
+ * assignment routed to that expert whose inverse entry points back at the row, so no assignment
+ * is held twice); at its end, a kernel that checks the canaries.  A failed check sets
+ * JMOE_DEV_BAD_TABLE or JMOE_DEV_CANARY in the status word (first error wins) and traps nothing.
+ * Host only; not thread-safe.
+ *
+ * jamba_moe_debug_corrupt — test hook for those checks: the next MoE forward call (one shot)
+ * corrupts its own state from the host, with in-bounds copies that no kernel can turn into a
+ * memory fault:
+ *   JMOE_CORRUPT_ROUTE_ID  after the router, routing id 0 := 0x7F7F7F7F (out of range: the
+ *                          permutation kernel skips it and reports JMOE_DEV_BAD_INDEX);
+ *   JMOE_CORRUPT_PERM_ROW  after the permutation, permuted row 1 := permuted row 0 (an assignment
+ *                          held twice: the table check reports JMOE_DEV_BAD_TABLE);
+ *   JMOE_CORRUPT_CANARY    before the final check, one byte of a guard gap (JMOE_DEV_CANARY).
+ * The output of that call is not valid.  0 cancels a pending corruption.  Host only.
+ */
+enum { JMOE_CORRUPT_NONE = 0, JMOE_CORRUPT_ROUTE_ID = 1, JMOE_CORRUPT_PERM_ROW = 2, JMOE_CORRUPT_CANARY = 3 };
+int jamba_moe_debug_checks(int on);
+int jamba_moe_debug_corrupt(int what);
+
+/*
  * jamba_moe_forward_noalloc — jamba_moe_forward on the decode (weight-streaming) path for callers
  * that cannot allocate device memory: code running inside a memory pool it does not own, a
  * serving process that must not call cudaMalloc after start-up (it synchronises the device and
@@ -264,6 +291,56 @@ size_t jamba_moe_noalloc_scratch_needed(int64_t T, int64_t d, int64_t ffn);
  * if the lookup or the 4-byte copy fails.  Allocates nothing.
  */
 int jamba_moe_noalloc_read_device_status(void* stream);
+
+/*
+ * Expert parallelism over G ranks (one GPU each; Jamba-1.5 paper, "Model Architecture": with
+ * ExpertsInt8, Jamba-1.5-Large is served on one machine of eight 80 GB GPUs; "Training
+ * Infrastructure": expert parallelism).  Rank g (0 <= g < G, G divides 16) holds the int8
+ * weights of experts [g*16/G, (g+1)*16/G) only, and its own batch of T tokens.  One layer call:
+ *
+ *   1. jamba_moe_ep_dispatch     router + permutation of the rank's tokens; rows of x packed in
+ *                                send order (grouped by destination rank, then expert, then token)
+ *   2. the caller's all-to-all   of send_counts, then of send_x / send_expert / send_w with those
+ *                                counts (e.g. torch.distributed.all_to_all_single over NCCL)
+ *   3. jamba_moe_ep_experts      the rank's experts on the N rows it received
+ *   4. the caller's all-to-all   of `out` back, in reverse, into a buffer `ret` in send order
+ *   5. jamba_moe_ep_combine      y[t] = bf16(ret[pos[t][0]] + ret[pos[t][1]])
+ *
+ * The rows cross the interconnect once each way; y equals jamba_moe_forward's up to the choice of
+ * expert path (both are within the same tolerance of the exact layer), the two slots being added
+ * in the same fixed order.
+ *
+ * jamba_moe_ep_dispatch — x bf16 [T][d], router as in jamba_moe_forward; n_ranks = G.  Writes
+ * send_x bf16 [T*2][d], send_expert int32 [T*2] (expert index local to the destination rank),
+ * send_w fp32 [T*2] (routing weight), send_counts int32 [G] (rows for each rank, in rank order:
+ * the first send_counts[0] rows go to rank 0, ...), pos int32 [T][2] (the send row of each
+ * assignment) and, if given, topk_ids / topk_w.  Only the first sum(send_counts) = 2T rows are
+ * written.  T = 0 writes zero counts.  workspace: jamba_moe_ep_dispatch_workspace_size bytes.
+ */
+size_t jamba_moe_ep_dispatch_workspace_size(int64_t T, int64_t d, int n_experts, int top_k);
+int jamba_moe_ep_dispatch(const uint16_t* x, const float* router_W, const float* router_bias, int64_t T, int64_t d,
+                          int n_experts, int top_k, int n_ranks, uint16_t* send_x, int32_t* send_expert,
+                          float* send_w, int32_t* send_counts, int32_t* pos, int32_t* topk_ids, float* topk_w,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * jamba_moe_ep_experts — the rank's n_local experts on N received rows: xr bf16 [N][d],
+ * expert int32 [N] in [0, n_local) (other values are skipped and reported as JMOE_DEV_BAD_INDEX in
+ * the workspace status word), w fp32 [N]; Q1, Q3 int8 [n_local][ffn][d], Q2 int8 [n_local][d][ffn]
+ * with their scales.  out fp32 [N][d]: out[n] = w[n] * E_expert[n](xr[n]) with the numerics of
+ * jamba_moe_forward (exact int8 -> bf16, fp32 accumulation, bf16 SwiGLU intermediate).  path as in
+ * jamba_moe_forward_path (AUTO: weight streaming when the rows per local expert are few).
+ * workspace: jamba_moe_ep_experts_workspace_size(N, d, ffn) bytes; N = 0 is a no-op.
+ */
+size_t jamba_moe_ep_experts_workspace_size(int64_t N, int64_t d, int64_t ffn);
+int jamba_moe_ep_experts(const uint16_t* xr, const int32_t* expert, const float* w, int64_t N, int64_t d, int64_t ffn,
+                         int n_local, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                         const int8_t* Q2, const float* S2, float* out, void* workspace, size_t workspace_bytes,
+                         void* stream, int path);
+
+/* jamba_moe_ep_combine — ret fp32 [T*2][d] (the outputs back in send order), pos from the
+ * dispatch: y bf16 [T][d] = bf16(ret[pos[t][0]] + ret[pos[t][1]]), slot 0 then slot 1. */
+int jamba_moe_ep_combine(const float* ret, const int32_t* pos, int64_t T, int64_t d, uint16_t* y, void* stream);
 
 /*
  * Kernel timing (for the benchmark's roofline figures).

@@ -89,6 +89,22 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                             vp, c_int]
     lib.jamba_moe_debug_skip_copy.restype = c_int
     lib.jamba_moe_debug_skip_copy.argtypes = [c_int]
+    lib.jamba_moe_ep_dispatch_workspace_size.restype = sz
+    lib.jamba_moe_ep_dispatch_workspace_size.argtypes = [i64, i64, c_int, c_int]
+    lib.jamba_moe_ep_dispatch.restype = c_int
+    lib.jamba_moe_ep_dispatch.argtypes = [vp, vp, vp, i64, i64, c_int, c_int, c_int, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                          vp]
+    lib.jamba_moe_ep_experts_workspace_size.restype = sz
+    lib.jamba_moe_ep_experts_workspace_size.argtypes = [i64, i64, i64]
+    lib.jamba_moe_ep_experts.restype = c_int
+    lib.jamba_moe_ep_experts.argtypes = [vp, vp, vp, i64, i64, i64, c_int, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                         c_int]
+    lib.jamba_moe_ep_combine.restype = c_int
+    lib.jamba_moe_ep_combine.argtypes = [vp, vp, i64, i64, vp, vp]
+    lib.jamba_moe_debug_checks.restype = c_int
+    lib.jamba_moe_debug_checks.argtypes = [c_int]
+    lib.jamba_moe_debug_corrupt.restype = c_int
+    lib.jamba_moe_debug_corrupt.argtypes = [c_int]
     lib.jamba_moe_kernel_name.restype = ctypes.c_char_p
     lib.jamba_moe_kernel_name.argtypes = [c_int]
     _lib = lib
@@ -435,6 +451,129 @@ def jamba_moe_read_device_status(workspace: torch.Tensor, stream: Optional[torch
 def jamba_moe_debug_skip_copy(on: bool) -> None:
     """Test hook (see include/jmoe.h): make one tensor-core pipeline wait run out on purpose."""
     load_library().jamba_moe_debug_skip_copy(1 if on else 0)
+
+
+def jamba_moe_ep_dispatch_workspace_size(T: int, d: int, n_experts: int = N_EXPERTS, top_k: int = TOP_K) -> int:
+    return int(load_library().jamba_moe_ep_dispatch_workspace_size(T, d, n_experts, top_k))
+
+
+def jamba_moe_ep_experts_workspace_size(N: int, d: int, ffn: int) -> int:
+    return int(load_library().jamba_moe_ep_experts_workspace_size(N, d, ffn))
+
+
+def jamba_moe_ep_dispatch(x: torch.Tensor, router_W: torch.Tensor, router_bias: Optional[torch.Tensor], n_ranks: int,
+                          workspace: Optional[torch.Tensor] = None, stream: Optional[torch.cuda.Stream] = None):
+    """Expert-parallel step 1 (see include/jmoe.h): route this rank's tokens x [T][d] and pack
+    their rows by destination rank.  Returns a dict: send_x bf16 [2T][d], send_expert int32 [2T]
+    (expert index local to its rank), send_w fp32 [2T], send_counts int32 [n_ranks], pos int32
+    [T][2], topk_ids int32 [T][2], topk_w fp32 [T][2], and the workspace (device status word)."""
+    lib = load_library()
+    _check(x, "x", torch.bfloat16)
+    T, d = x.shape
+    E = router_W.shape[0]
+    _check(router_W, "router_W", torch.float32, (E, d))
+    if router_bias is not None:
+        _check(router_bias, "router_bias", torch.float32, (E,))
+    dev = x.device
+    out = dict(send_x=torch.empty((T * TOP_K, d), dtype=torch.bfloat16, device=dev),
+               send_expert=torch.empty(T * TOP_K, dtype=torch.int32, device=dev),
+               send_w=torch.empty(T * TOP_K, dtype=torch.float32, device=dev),
+               send_counts=torch.empty(n_ranks, dtype=torch.int32, device=dev),
+               pos=torch.empty((T, TOP_K), dtype=torch.int32, device=dev),
+               topk_ids=torch.empty((T, TOP_K), dtype=torch.int32, device=dev),
+               topk_w=torch.empty((T, TOP_K), dtype=torch.float32, device=dev))
+    need = int(lib.jamba_moe_ep_dispatch_workspace_size(T, d, E, TOP_K))
+    if need == 0:
+        raise JmoeError(2, "jamba_moe_ep_dispatch_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _check(workspace, "workspace", torch.uint8)
+    p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    _one_device(x, router_W=router_W, router_bias=router_bias, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_ep_dispatch(x.data_ptr(), router_W.data_ptr(), p(router_bias), T, d, E, TOP_K, int(n_ranks),
+                                       out["send_x"].data_ptr(), out["send_expert"].data_ptr(),
+                                       out["send_w"].data_ptr(), out["send_counts"].data_ptr(), out["pos"].data_ptr(),
+                                       out["topk_ids"].data_ptr(), out["topk_w"].data_ptr(), workspace.data_ptr(),
+                                       workspace.numel(), _stream_ptr(stream, dev))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_ep_dispatch")
+    out["workspace"] = workspace
+    return out
+
+
+def jamba_moe_ep_experts(xr: torch.Tensor, expert: torch.Tensor, w: torch.Tensor, Q1: torch.Tensor, S1: torch.Tensor,
+                         Q3: torch.Tensor, S3: torch.Tensor, Q2: torch.Tensor, S2: torch.Tensor,
+                         out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None, path: int = PATH_AUTO) -> torch.Tensor:
+    """Expert-parallel step 3: this rank's experts (Q1, Q3 int8 [n_local][ffn][d], Q2 int8
+    [n_local][d][ffn] and scales) on the N received rows xr [N][d] with their local expert index
+    and routing weight.  Returns out fp32 [N][d] = w * E_expert(xr)."""
+    lib = load_library()
+    _check(xr, "xr", torch.bfloat16)
+    N, d = xr.shape
+    n_local, ffn = Q1.shape[0], Q1.shape[1]
+    _check(expert, "expert", torch.int32, (N,))
+    _check(w, "w", torch.float32, (N,))
+    _check(Q1, "Q1", torch.int8, (n_local, ffn, d))
+    _check(Q3, "Q3", torch.int8, (n_local, ffn, d))
+    _check(Q2, "Q2", torch.int8, (n_local, d, ffn))
+    _check(S1, "S1", torch.float32, (n_local, ffn))
+    _check(S3, "S3", torch.float32, (n_local, ffn))
+    _check(S2, "S2", torch.float32, (n_local, d))
+    if out is None:
+        out = torch.empty((N, d), dtype=torch.float32, device=xr.device)
+    _check(out, "out", torch.float32, (N, d))
+    need = int(lib.jamba_moe_ep_experts_workspace_size(N, d, ffn))
+    if need == 0:
+        raise JmoeError(2, "jamba_moe_ep_experts_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=xr.device)
+    _check(workspace, "workspace", torch.uint8)
+    dev = _one_device(xr, expert=expert, w=w, Q1=Q1, S1=S1, Q3=Q3, S3=S3, Q2=Q2, S2=S2, out=out, workspace=workspace)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_ep_experts(xr.data_ptr(), expert.data_ptr(), w.data_ptr(), N, d, ffn, n_local,
+                                      Q1.data_ptr(), S1.data_ptr(), Q3.data_ptr(), S3.data_ptr(), Q2.data_ptr(),
+                                      S2.data_ptr(), out.data_ptr(), workspace.data_ptr(), workspace.numel(),
+                                      _stream_ptr(stream, dev), int(path))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_ep_experts")
+    return out
+
+
+def jamba_moe_ep_combine(ret: torch.Tensor, pos: torch.Tensor, y: Optional[torch.Tensor] = None,
+                         stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Expert-parallel step 5: y bf16 [T][d] = bf16(ret[pos[t][0]] + ret[pos[t][1]])."""
+    lib = load_library()
+    _check(ret, "ret", torch.float32)
+    _check(pos, "pos", torch.int32)
+    T, d = pos.shape[0], ret.shape[1]
+    _check(ret, "ret", torch.float32, (T * TOP_K, d))
+    _check(pos, "pos", torch.int32, (T, TOP_K))
+    if y is None:
+        y = torch.empty((T, d), dtype=torch.bfloat16, device=ret.device)
+    _check(y, "y", torch.bfloat16, (T, d))
+    dev = _one_device(ret, pos=pos, y=y)
+    with torch.cuda.device(dev):
+        st = lib.jamba_moe_ep_combine(ret.data_ptr(), pos.data_ptr(), T, d, y.data_ptr(), _stream_ptr(stream, dev))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_ep_combine")
+    return y
+
+
+CORRUPT_NONE, CORRUPT_ROUTE_ID, CORRUPT_PERM_ROW, CORRUPT_CANARY = 0, 1, 2, 3
+
+
+def jamba_moe_debug_checks(on: bool) -> None:
+    """Debug checks of every MoE forward call (see include/jmoe.h): routing tables and canaries."""
+    load_library().jamba_moe_debug_checks(1 if on else 0)
+
+
+def jamba_moe_debug_corrupt(what: int) -> None:
+    """Test hook (see include/jmoe.h): the next MoE forward call corrupts its own state, in bounds."""
+    st = load_library().jamba_moe_debug_corrupt(int(what))
+    if st != 0:
+        raise JmoeError(st, "jamba_moe_debug_corrupt")
 
 
 def jamba_moe_timing_start(max_launches: int) -> None:

@@ -14,7 +14,7 @@ cudaError_t launch_router(const uint16_t* x, const float* Wr, const float* bias,
 cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
                            cudaStream_t st);
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
-                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid);
+                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid, int k_div = kTopK);
 cudaError_t launch_gemv13_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const uint16_t* W1,
                                 const uint16_t* W3, uint16_t* h, int64_t T, int64_t d, int64_t F, cudaStream_t st);
 cudaError_t launch_gemv2_bf16w(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const uint16_t* W2,
@@ -27,7 +27,7 @@ cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_
                                cudaStream_t st);
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
-                          int64_t F, cudaStream_t st);
+                          int64_t F, cudaStream_t st, int k_div = kTopK);
 cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
                          const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
                          cudaStream_t st);
@@ -61,6 +61,11 @@ cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h
                             const float* S2, const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F,
                             cudaStream_t st);
 
+cudaError_t launch_tables_check(WsHeader* hdr, const int32_t* ids, const int32_t* perm, const int32_t* inv, int64_t TK,
+                                int64_t rows_cap, cudaStream_t st);
+cudaError_t launch_canary_fill(uint8_t* ws, const GuardGaps& g, cudaStream_t st);
+cudaError_t launch_canary_check(const uint8_t* ws, const GuardGaps& g, WsHeader* hdr, cudaStream_t st);
+
 namespace {
 
 constexpr int64_t kMaxT = int64_t(1) << 20;
@@ -72,7 +77,27 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct Layout {
     int64_t rows_cap;  // permuted rows incl. per-expert padding
     size_t hdr, ids, wts, inv, perm, x_perm, h, slots, total;
+    GuardGaps guards;  // a canary gap after every region
 };
+
+// Region allocator of the workspace layouts: 256-byte aligned regions, each followed by a guard
+// gap of kGuardBytes (checked for overwrites when the debug checks are on).
+struct Regions {
+    size_t off = 0;
+    GuardGaps g{};
+    size_t take(size_t bytes) {
+        const size_t at = off;
+        off = (off + bytes + 255) & ~size_t(255);
+        if (g.n < kMaxGuards) g.off[g.n++] = off;
+        off += kGuardBytes;
+        return at;
+    }
+};
+
+// Test hooks (host-side state, not thread-safe): debug checks on every forward call, and a one-shot
+// corruption of the next call's routing state, made from the host with in-bounds copies.
+int g_debug_checks = 0;
+int g_corrupt = 0;  // JMOE_CORRUPT_*
 
 bool shape_ok(int64_t T, int64_t d, int64_t F, int E, int K) {
     if (E != kExperts || K != kTopK) return false;
@@ -86,25 +111,53 @@ Layout make_layout(int64_t T, int64_t d, int64_t F) {
     Layout L{};
     const int64_t TK = T * kTopK;
     L.rows_cap = (TK + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
-    size_t off = 0;
-    L.hdr = off;
-    off = align256(off + kHeaderBytes);
-    L.ids = off;
-    off = align256(off + sizeof(int32_t) * TK);
-    L.wts = off;
-    off = align256(off + sizeof(float) * TK);
-    L.inv = off;
-    off = align256(off + sizeof(int32_t) * TK);
-    L.perm = off;
-    off = align256(off + sizeof(int32_t) * L.rows_cap);
-    L.x_perm = off;
-    off = align256(off + sizeof(uint16_t) * L.rows_cap * d);
-    L.h = off;
-    off = align256(off + sizeof(uint16_t) * L.rows_cap * F);
-    L.slots = off;
-    off = align256(off + sizeof(float) * TK * d);
-    L.total = off;
+    Regions R;
+    L.hdr = R.take(kHeaderBytes);
+    L.ids = R.take(sizeof(int32_t) * TK);
+    L.wts = R.take(sizeof(float) * TK);
+    L.inv = R.take(sizeof(int32_t) * TK);
+    L.perm = R.take(sizeof(int32_t) * L.rows_cap);
+    L.x_perm = R.take(sizeof(uint16_t) * L.rows_cap * d);
+    L.h = R.take(sizeof(uint16_t) * L.rows_cap * F);
+    L.slots = R.take(sizeof(float) * TK * d);
+    L.total = R.off;
+    L.guards = R.g;
     return L;
+}
+
+// The debug-check and corruption steps of a MoE forward call, at the points the call reaches.
+enum Step { kAtStart, kAfterRouter, kAfterPermute, kAtEnd };
+cudaError_t debug_step(Step at, char* ws, const GuardGaps& guards, WsHeader* hdr, int32_t* ids, const int32_t* perm,
+                       const int32_t* inv, int64_t TK, int64_t rows_cap, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+    switch (at) {
+        case kAtStart:
+            if (g_debug_checks) e = launch_canary_fill(w8, guards, st);
+            break;
+        case kAfterRouter:
+            if (g_corrupt == JMOE_CORRUPT_ROUTE_ID) {  // routing id of assignment 0 := 0x7F7F7F7F
+                g_corrupt = 0;
+                e = cudaMemsetAsync(ids, 0x7F, sizeof(int32_t), st);
+            }
+            break;
+        case kAfterPermute:
+            if (g_corrupt == JMOE_CORRUPT_PERM_ROW) {  // permuted row 1 := permuted row 0
+                g_corrupt = 0;
+                e = cudaMemcpyAsync(const_cast<int32_t*>(perm) + 1, perm, sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                                    st);
+            }
+            if (e == cudaSuccess && g_debug_checks) e = launch_tables_check(hdr, ids, perm, inv, TK, rows_cap, st);
+            break;
+        case kAtEnd:
+            if (g_corrupt == JMOE_CORRUPT_CANARY && guards.n > 1) {  // one byte of the second guard gap
+                g_corrupt = 0;
+                e = cudaMemsetAsync(w8 + guards.off[1] + 17, 0x5A, 1, st);
+            }
+            if (e == cudaSuccess && g_debug_checks) e = launch_canary_check(w8, guards, hdr, st);
+            break;
+    }
+    return e;
 }
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -215,17 +268,23 @@ int forward_impl(const uint16_t* x, const float* router_W, const float* router_b
     const uint16_t* B3 = static_cast<const uint16_t*>(W3);
     const uint16_t* B2 = static_cast<const uint16_t*>(W2);
 
-    cudaError_t e;
+    const int64_t TK = T * kTopK;
+    cudaError_t e = debug_step(kAtStart, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st);
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_ROUTER, st);
         e = launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st);
     }
     if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (debug_step(kAfterRouter, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st) != cudaSuccess)
+        return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
         e = launch_permute(ids, T, hdr, perm, inv, st);
     }
     if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (debug_step(kAfterPermute, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st) != cudaSuccess)
+        return JMOE_ERR_CUDA;
     if (path == JMOE_PATH_GEMV) {
         {
             TimedLaunch t(JMOE_KERNEL_GEMV13, st);
@@ -262,7 +321,8 @@ int forward_impl(const uint16_t* x, const float* router_W, const float* router_b
         TimedLaunch t(JMOE_KERNEL_COMBINE, st);
         e = launch_combine(slots, T, d, y, st, sms);
     }
-    return to_status(e);
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    return to_status(debug_step(kAtEnd, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st));
 }
 
 }  // namespace
@@ -357,18 +417,15 @@ namespace {
 struct LayoutF8 {
     int64_t rows_cap;
     size_t hdr, ids, wts, inv, perm, x8, sx, x8_perm, h, h8, sh, slots, total;
+    GuardGaps guards;
 };
 
 LayoutF8 make_layout_f8(int64_t T, int64_t d, int64_t F) {
     LayoutF8 L{};
     const int64_t TK = T * kTopK;
     L.rows_cap = (TK + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
-    size_t off = 0;
-    auto take = [&](size_t bytes) {
-        const size_t at = off;
-        off = align256(off + bytes);
-        return at;
-    };
+    Regions R;
+    auto take = [&](size_t bytes) { return R.take(bytes); };
     L.hdr = take(kHeaderBytes);
     L.ids = take(sizeof(int32_t) * TK);
     L.wts = take(sizeof(float) * TK);
@@ -381,7 +438,8 @@ LayoutF8 make_layout_f8(int64_t T, int64_t d, int64_t F) {
     L.h8 = take((size_t)L.rows_cap * F);
     L.sh = take(sizeof(float) * L.rows_cap);
     L.slots = take(sizeof(float) * TK * d);
-    L.total = off;
+    L.total = R.off;
+    L.guards = R.g;
     return L;
 }
 
@@ -420,17 +478,23 @@ int forward_f8(const uint16_t* x, const float* router_W, const float* router_bia
     const int sms = num_sms_current();
     if (path == JMOE_PATH_AUTO) path = (T <= kGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
 
-    cudaError_t e;
+    const int64_t TK = T * kTopK;
+    cudaError_t e = debug_step(kAtStart, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st);
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_ROUTER, st);
         e = launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st);
     }
     if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (debug_step(kAfterRouter, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st) != cudaSuccess)
+        return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
         e = launch_permute(ids, T, hdr, perm, inv, st);
     }
     if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (debug_step(kAfterPermute, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st) != cudaSuccess)
+        return JMOE_ERR_CUDA;
     {
         TimedLaunch t(JMOE_KERNEL_ACT_QUANT, st);  // per-token E4M3 activations
         e = launch_quantize_fp8(x, T, d, x8, sx, nullptr, nullptr, st, sms);
@@ -476,8 +540,12 @@ int forward_f8(const uint16_t* x, const float* router_W, const float* router_bia
         }
         if (e != cudaSuccess) return JMOE_ERR_CUDA;
     }
-    TimedLaunch t(JMOE_KERNEL_COMBINE, st);
-    return to_status(launch_combine(slots, T, d, y, st, sms));
+    {
+        TimedLaunch t(JMOE_KERNEL_COMBINE, st);
+        e = launch_combine(slots, T, d, y, st, sms);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    return to_status(debug_step(kAtEnd, ws, L.guards, hdr, ids, perm, inv, TK, L.rows_cap, st));
 }
 
 }  // namespace
@@ -574,8 +642,21 @@ const char* jamba_moe_status_string(int status) {
         case JMOE_DEV_TIMEOUT: return "a kernel gave up waiting on a pipeline barrier";
         case JMOE_DEV_BAD_INDEX: return "a kernel saw an out-of-range routing index";
         case JMOE_ERR_ALIGN: return "a pointer is not 16-byte aligned";
+        case JMOE_DEV_BAD_TABLE: return "a debug check found inconsistent routing tables";
+        case JMOE_DEV_CANARY: return "a debug check found a workspace guard gap overwritten";
         default: return "unknown status";
     }
+}
+
+int jamba_moe_debug_checks(int on) {
+    g_debug_checks = on ? 1 : 0;
+    return JMOE_OK;
+}
+
+int jamba_moe_debug_corrupt(int what) {
+    if (what < 0 || what > JMOE_CORRUPT_CANARY) return JMOE_ERR_SHAPE;
+    g_corrupt = what;
+    return JMOE_OK;
 }
 
 int jamba_moe_timing_start(int max_launches) {
@@ -625,6 +706,174 @@ const char* jamba_moe_kernel_name(int kind) {
     static const char* names[JMOE_KERNEL_KINDS] = {"quantize", "router", "permute", "gather", "gemv13",
                                                    "gemv2", "gemm13", "gemm2", "combine", "act_quant"};
     return (kind >= 0 && kind < JMOE_KERNEL_KINDS) ? names[kind] : "unknown";
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- expert parallelism (ep.cu)
+namespace jmoe {
+cudaError_t launch_permute_tk(const int32_t* ids, int64_t TK, int n_valid, WsHeader* hdr, int32_t* perm, int32_t* inv,
+                              cudaStream_t st);
+cudaError_t launch_ep_pack(const uint16_t* x, const WsHeader* hdr, const int32_t* perm, const float* wts, int64_t d,
+                           int64_t rows_cap, int experts_per_rank, int n_ranks, uint16_t* send_x, int32_t* send_e,
+                           float* send_w, int32_t* pos, int32_t* send_counts, cudaStream_t st, int num_sms);
+cudaError_t launch_ep_combine(const float* ret, const int32_t* pos, int64_t T, int64_t d, uint16_t* y, cudaStream_t st,
+                              int num_sms);
+}  // namespace jmoe
+
+namespace {
+
+bool ranks_ok(int n_ranks) { return n_ranks >= 1 && n_ranks <= kExperts && kExperts % n_ranks == 0; }
+
+// Dispatch workspace: routing tables of the rank's own tokens.
+Layout make_layout_ep_dispatch(int64_t T) {
+    Layout L{};
+    const int64_t TK = T * kTopK;
+    L.rows_cap = (TK + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
+    Regions R;
+    L.hdr = R.take(kHeaderBytes);
+    L.ids = R.take(sizeof(int32_t) * TK);
+    L.wts = R.take(sizeof(float) * TK);
+    L.inv = R.take(sizeof(int32_t) * TK);
+    L.perm = R.take(sizeof(int32_t) * L.rows_cap);
+    L.total = R.off;
+    L.guards = R.g;
+    return L;
+}
+
+// Expert workspace: the received rows' routing tables, permuted rows and SwiGLU intermediate.
+Layout make_layout_ep_experts(int64_t N, int64_t d, int64_t F) {
+    Layout L{};
+    L.rows_cap = (N + int64_t(kExperts) * (kRowPad - 1) + kRowPad - 1) / kRowPad * kRowPad;
+    Regions R;
+    L.hdr = R.take(kHeaderBytes);
+    L.inv = R.take(sizeof(int32_t) * (N > 0 ? N : 1));
+    L.perm = R.take(sizeof(int32_t) * L.rows_cap);
+    L.x_perm = R.take(sizeof(uint16_t) * L.rows_cap * d);
+    L.h = R.take(sizeof(uint16_t) * L.rows_cap * F);
+    L.total = R.off;
+    L.guards = R.g;
+    return L;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t jamba_moe_ep_dispatch_workspace_size(int64_t T, int64_t d, int n_experts, int top_k) {
+    if (!shape_ok(T, d, 128, n_experts, top_k)) return 0;
+    return make_layout_ep_dispatch(T).total;
+}
+
+int jamba_moe_ep_dispatch(const uint16_t* x, const float* router_W, const float* router_bias, int64_t T, int64_t d,
+                          int n_experts, int top_k, int n_ranks, uint16_t* send_x, int32_t* send_expert,
+                          float* send_w, int32_t* send_counts, int32_t* pos, int32_t* topk_ids, float* topk_w,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+    if (!shape_ok(T, d, 128, n_experts, top_k) || !ranks_ok(n_ranks)) return JMOE_ERR_SHAPE;
+    if (!send_counts) return JMOE_ERR_NULL;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) return to_status(cudaMemsetAsync(send_counts, 0, sizeof(int32_t) * n_ranks, st));
+    if (!x || !router_W || !send_x || !send_expert || !send_w || !pos || !workspace) return JMOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(router_W) || !aligned16(send_x)) return JMOE_ERR_ALIGN;
+    const void* ptrs4[] = {router_bias, send_expert, send_w, send_counts, pos, topk_ids, topk_w};
+    for (const void* p : ptrs4)
+        if (reinterpret_cast<uintptr_t>(p) & 3) return JMOE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return JMOE_ERR_WORKSPACE;
+    const Layout L = make_layout_ep_dispatch(T);
+    if (workspace_bytes < L.total) return JMOE_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+    int32_t* ids = reinterpret_cast<int32_t*>(ws + L.ids);
+    float* wts = reinterpret_cast<float*>(ws + L.wts);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    cudaError_t e;
+    {
+        TimedLaunch t(JMOE_KERNEL_ROUTER, st);
+        e = launch_router(x, router_W, router_bias, T, d, ids, wts, topk_ids, topk_w, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
+        e = launch_permute(ids, T, hdr, perm, inv, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    TimedLaunch t(JMOE_KERNEL_GATHER, st);
+    return to_status(launch_ep_pack(x, hdr, perm, wts, d, L.rows_cap, kExperts / n_ranks, n_ranks, send_x, send_expert,
+                                    send_w, pos, send_counts, st, num_sms_current()));
+}
+
+size_t jamba_moe_ep_experts_workspace_size(int64_t N, int64_t d, int64_t ffn) {
+    if (!shape_ok(N, d, ffn, kExperts, kTopK)) return 0;
+    return make_layout_ep_experts(N, d, ffn).total;
+}
+
+int jamba_moe_ep_experts(const uint16_t* xr, const int32_t* expert, const float* w, int64_t N, int64_t d, int64_t ffn,
+                         int n_local, const int8_t* Q1, const float* S1, const int8_t* Q3, const float* S3,
+                         const int8_t* Q2, const float* S2, float* out, void* workspace, size_t workspace_bytes,
+                         void* stream, int path) {
+    if (!shape_ok(N, d, ffn, kExperts, kTopK) || n_local < 1 || n_local > kExperts) return JMOE_ERR_SHAPE;
+    if (path != JMOE_PATH_AUTO && path != JMOE_PATH_GEMV && path != JMOE_PATH_GEMM) return JMOE_ERR_SHAPE;
+    if (N == 0) return JMOE_OK;
+    if (!xr || !expert || !w || !Q1 || !S1 || !Q3 || !S3 || !Q2 || !S2 || !out || !workspace) return JMOE_ERR_NULL;
+    const void* ptrs16[] = {xr, Q1, Q3, Q2, out};
+    for (const void* p : ptrs16)
+        if (!aligned16(p)) return JMOE_ERR_ALIGN;
+    const void* ptrs4[] = {expert, w, S1, S3, S2};
+    for (const void* p : ptrs4)
+        if (reinterpret_cast<uintptr_t>(p) & 3) return JMOE_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255) return JMOE_ERR_WORKSPACE;
+    const Layout L = make_layout_ep_experts(N, d, ffn);
+    if (workspace_bytes < L.total) return JMOE_ERR_WORKSPACE;
+    char* ws = static_cast<char*>(workspace);
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws + L.hdr);
+    int32_t* inv = reinterpret_cast<int32_t*>(ws + L.inv);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    uint16_t* x_perm = reinterpret_cast<uint16_t*>(ws + L.x_perm);
+    uint16_t* h = reinterpret_cast<uint16_t*>(ws + L.h);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // one assignment per received row (k_div = 1); the GEMV pass width follows the rows per local
+    // expert, given to the launcher as the token count whose K assignments spread over 16 experts
+    const int64_t rows_per_expert = (N + n_local - 1) / n_local;
+    const int64_t T_equiv = (rows_per_expert * kExperts + kTopK - 1) / kTopK;
+    if (path == JMOE_PATH_AUTO) path = (T_equiv <= kGemvMaxTokens) ? JMOE_PATH_GEMV : JMOE_PATH_GEMM;
+    cudaError_t e;
+    {
+        TimedLaunch t(JMOE_KERNEL_PERMUTE, st);
+        e = launch_permute_tk(expert, N, n_local, hdr, perm, inv, st);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    if (path == JMOE_PATH_GEMV) {
+        {
+            TimedLaunch t(JMOE_KERNEL_GEMV13, st);
+            e = launch_gemv13(hdr, perm, xr, Q1, S1, Q3, S3, h, T_equiv, d, ffn, st, 1);
+        }
+        if (e != cudaSuccess) return JMOE_ERR_CUDA;
+        TimedLaunch t(JMOE_KERNEL_GEMV2, st);
+        return to_status(launch_gemv2(hdr, perm, h, Q2, S2, w, out, T_equiv, d, ffn, st));
+    }
+    {
+        TimedLaunch t(JMOE_KERNEL_GATHER, st);
+        e = launch_gather(xr, perm, hdr, d, L.rows_cap, x_perm, st, num_sms_current(), true, 1);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    {
+        TimedLaunch t(JMOE_KERNEL_GEMM13, st);
+        e = launch_gemm13(hdr, perm, x_perm, Q1, S1, Q3, S3, h, L.rows_cap, d, ffn, st, n_local);
+    }
+    if (e != cudaSuccess) return JMOE_ERR_CUDA;
+    TimedLaunch t(JMOE_KERNEL_GEMM2, st);
+    return to_status(launch_gemm2(hdr, perm, h, Q2, S2, w, out, L.rows_cap, d, ffn, st, n_local, nullptr));
+}
+
+int jamba_moe_ep_combine(const float* ret, const int32_t* pos, int64_t T, int64_t d, uint16_t* y, void* stream) {
+    if (!shape_ok(T, d, 128, kExperts, kTopK)) return JMOE_ERR_SHAPE;
+    if (T == 0) return JMOE_OK;
+    if (!ret || !pos || !y) return JMOE_ERR_NULL;
+    if (!aligned16(ret) || !aligned16(y) || (reinterpret_cast<uintptr_t>(pos) & 3)) return JMOE_ERR_ALIGN;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    TimedLaunch t(JMOE_KERNEL_COMBINE, st);
+    return to_status(launch_ep_combine(ret, pos, T, d, y, st, num_sms_current()));
 }
 
 }  // extern "C"

@@ -19,7 +19,8 @@ constexpr int kRowPad = 128;  // each expert's segment of permuted rows starts o
 // The first kHeaderBytes of the workspace hold the routing tables the kernels exchange.
 struct WsHeader {
     uint32_t status;              // JMOE_OK or a JMOE_DEV_* code (first error wins)
-    uint32_t pad0[15];
+    int32_t sched[2];             // tile counters of the two tensor-core GEMMs (dynamic scheduling)
+    uint32_t pad0[13];
     int32_t counts[kExperts];     // tokens routed to each expert
     int32_t seg_start[kExperts + 1];  // first permuted row of each expert (multiple of kRowPad)
     int32_t pad1[15];
@@ -28,11 +29,28 @@ struct WsHeader {
     int32_t touched[kExperts];    // experts with at least one token, ascending
     int32_t n_touched;
     int32_t pad3[15];
+    // the touched experts split by count (decode path: one pass of 8 tokens, or passes of 16)
+    int32_t few[kExperts];        // 1 .. kFewTokens tokens, ascending
+    int32_t n_few;
+    int32_t pad4[15];
+    int32_t many[kExperts];       // more than kFewTokens tokens, ascending
+    int32_t n_many;
+    int32_t pad5[15];
 };
+constexpr int kFewTokens = 8;
 constexpr size_t kHeaderBytes = 4096;
 static_assert(sizeof(WsHeader) <= kHeaderBytes, "header too large");
 
 __device__ __forceinline__ void set_status(WsHeader* h, uint32_t code) { atomicCAS(&h->status, 0u, code); }
+
+// Guard gaps of a workspace layout: kGuardBytes after each region, filled with a canary pattern
+// and checked when the debug checks are on (byte offsets from the workspace start).
+constexpr uint32_t kGuardBytes = 256;
+constexpr int kMaxGuards = 16;
+struct GuardGaps {
+    uint64_t off[kMaxGuards];
+    int n;
+};
 
 // ------------------------------------------------------------------ loads
 __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {

@@ -501,8 +501,6 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int g_skip_copy = 0;  // set by jamba_moe_debug_skip_copy (tests only)
-
 int band_for(int K) {
     // keep a band's activation tiles (band * 128 rows * K * 2 bytes) near 24 MB of L2
     const int64_t per_tile = (int64_t)kBM * K * 2;
@@ -533,45 +531,6 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
 }
 
 }  // namespace
-
-// h = SwiGLU(x_perm . Q1^T, x_perm . Q3^T) per expert segment; rows_cap = permuted-row capacity;
-// n_exp = experts held by Q1/Q3 (16, or 1 for the dense MLP).
-cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_perm, const int8_t* Q1,
-                          const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
-                          int64_t d, int64_t F, cudaStream_t st, int n_exp) {
-    CUtensorMap ta, tb0, tb1;
-    if (!make_map(&ta, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kBM, kBK,
-                  CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tb0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * F, d, 128, kBK,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_map(&tb1, Q3, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * F, d, 128, kBK,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    GemmArgs p{hdr,          perm,          S1,          S3,
-               nullptr,      h,             nullptr,     (int)d,
-               (int)F,       (int)(F / 128), band_for((int)d), g_skip_copy ? kTestMaxPolls : kMaxPolls,
-               g_skip_copy};
-    return launch_gemm_t<true, 256, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
-}
-
-// out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment, or, given y (the dense MLP, one
-// assignment per token), y[a / K] = bf16(p_a * S2 . (h_perm . Q2^T)).
-cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2, const float* S2,
-                         const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st,
-                         int n_exp, uint16_t* y) {
-    const int BN = (d % 256 == 0) ? 256 : 128;
-    CUtensorMap ta, tb0;
-    if (!make_map(&ta, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&tb0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * d, F, BN, kBK,
-                  CU_TENSOR_MAP_SWIZZLE_NONE))
-        return cudaErrorInvalidValue;
-    GemmArgs p{hdr,         perm,         S2,          nullptr,
-               wts,         nullptr,      out_slot,    (int)F,
-               (int)d,      (int)(d / BN), band_for((int)F), g_skip_copy ? kTestMaxPolls : kMaxPolls,
-               0,           y};
-    if (BN == 256) return launch_gemm_t<false, 256, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
-    return launch_gemm_t<false, 128, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
-}
 
 // The same two GEMMs with unquantized bf16 weights: the weight tiles are TMA-loaded in the
 // MMA's layout, nothing is converted, no scales are applied, and activations keep their k order.
@@ -648,11 +607,3 @@ cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h
 }
 
 }  // namespace jmoe
-
-// Test hook: while `on` is non-zero, the W1/W3 tensor-core GEMM's CTA 0 skips the copies of its
-// second K step, so the pipeline wait for them runs out (after a short bound) and the kernel must
-// report JMOE_DEV_TIMEOUT, release its resources and return.  Nothing faults or hangs.
-extern "C" int jamba_moe_debug_skip_copy(int on) {
-    jmoe::g_skip_copy = on ? 1 : 0;
-    return JMOE_OK;
-}

@@ -36,7 +36,10 @@ struct GemvArgs {
     int64_t K;             // reduction length: d (gemv13) or F (gemv2)
     int64_t N;             // weight rows per expert: F (gemv13) or d (gemv2)
     uint16_t* y_out;       // gemv2 of the dense MLP: y [T][d] in bf16, written instead of out_slot
+    int list;              // experts this launch serves: kAllTouched, kFewOnly or kManyOnly
+    int k_div;             // assignments per activation row of gemv13 (x row = assignment / k_div; 0: K)
 };
+enum { kAllTouched = 0, kFewOnly = 1, kManyOnly = 2 };
 
 // One k-step (16 consecutive k per lane) of weights for rows g and g+8: int8 codes fill one
 // 16-byte vector per row, bf16 weights two.
@@ -204,8 +207,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32,
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
     pdl_wait();
     const WsHeader* hdr = p.hdr;
-    if ((int)blockIdx.y >= hdr->n_touched) return;
-    const int e = hdr->touched[blockIdx.y];
+    const int n_list = p.list == kFewOnly ? hdr->n_few : (p.list == kManyOnly ? hdr->n_many : hdr->n_touched);
+    if ((int)blockIdx.y >= n_list) return;
+    const int e = (p.list == kFewOnly ? hdr->few : (p.list == kManyOnly ? hdr->many : hdr->touched))[blockIdx.y];
     const int m = hdr->counts[e];
     const int64_t row0 = hdr->seg_start[e];
     const int64_t j0 = (int64_t)blockIdx.x * kGemvRows;
@@ -219,7 +223,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32,
             const int nn = n < m ? n : 0;  // past the count: any valid row, its column is ignored
             if (kDual) {
                 const int32_t a = p.perm[row0 + nn];
-                rows[nt] = p.act + (int64_t)(a / kTopK) * p.K;
+                rows[nt] = p.act + (int64_t)(a / p.k_div) * p.K;
             } else {
                 rows[nt] = p.act + (row0 + nn) * p.K;
             }
@@ -262,17 +266,36 @@ static int gemv_nt(int64_t T) {
 static int gemv_nt_dense(int64_t T) { return T <= 8 ? 1 : (T <= 16 ? 2 : 4); }
 
 template <bool kDual, bool kW8>
-static cudaError_t launch_gemv_t(const GemvArgs& p, int nt, cudaStream_t st, int experts = kExperts) {
+static cudaError_t launch_gemv_nt(const GemvArgs& p, int nt, cudaStream_t st, int experts) {
     dim3 grid((unsigned)(p.N / kGemvRows), (unsigned)experts);
     if (nt == 1) return launch_pdl(gemv_kernel<1, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
     if (nt == 2) return launch_pdl(gemv_kernel<2, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
     return launch_pdl(gemv_kernel<4, kDual, kW8>, grid, dim3(kGemvWarps * 32), 0, st, p);
 }
 
+// Passes of 16 tokens (nt = 2) stream the weights slower than passes of 8 (nt = 1: more CTAs per
+// SM).  When the batch calls for 16-token passes, experts with at most 8 tokens take one launch of
+// the 8-token kernel and the others one launch of the 16-token kernel, so each expert's weights
+// are still streamed once.
+template <bool kDual, bool kW8>
+static cudaError_t launch_gemv_t(GemvArgs p, int nt, cudaStream_t st, int experts = kExperts) {
+    if (p.k_div <= 0) p.k_div = kTopK;
+    if (nt != 2 || experts != kExperts) {
+        p.list = kAllTouched;
+        return launch_gemv_nt<kDual, kW8>(p, nt, st, experts);
+    }
+    p.list = kFewOnly;
+    cudaError_t e = launch_gemv_nt<kDual, kW8>(p, 1, st, experts);
+    if (e != cudaSuccess) return e;
+    p.list = kManyOnly;
+    return launch_gemv_nt<kDual, kW8>(p, 2, st, experts);
+}
+
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
-                          int64_t F, cudaStream_t st) {
+                          int64_t F, cudaStream_t st, int k_div) {
     GemvArgs p{hdr, perm, x, Q1, Q3, S1, S3, nullptr, h, nullptr, d, F};
+    p.k_div = k_div;
     return launch_gemv_t<true, true>(p, gemv_nt(T), st);
 }
 

@@ -29,7 +29,7 @@ cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t
                            cudaStream_t st);
 cudaError_t launch_gemv13(const WsHeader* hdr, const int32_t* perm, const uint16_t* x, const int8_t* Q1,
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t T, int64_t d,
-                          int64_t F, cudaStream_t st);
+                          int64_t F, cudaStream_t st, int k_div = kTopK);
 cudaError_t launch_gemv2(const WsHeader* hdr, const int32_t* perm, const uint16_t* h, const int8_t* Q2,
                          const float* S2, const float* wts, float* out_slot, int64_t T, int64_t d, int64_t F,
                          cudaStream_t st);

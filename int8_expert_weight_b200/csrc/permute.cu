@@ -21,7 +21,7 @@ constexpr int kPermThreads = 1024;
 __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __restrict__ ids, int64_t TK,
                                                                WsHeader* __restrict__ hdr,
                                                                int32_t* __restrict__ perm,
-                                                               int32_t* __restrict__ inv) {
+                                                               int32_t* __restrict__ inv, int n_valid) {
     __shared__ int hist[kExperts];
     __shared__ int seg[kExperts + 1];
     __shared__ int base[kExperts];
@@ -31,12 +31,16 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
     pdl_wait();
     pdl_trigger();
     if (tid < kExperts) hist[tid] = 0;
-    if (tid == 0) hdr->status = 0;  // first kernel of a forward call to touch the header
+    if (tid == 0) {  // first kernel of a forward call to touch the header
+        hdr->status = 0;
+        hdr->sched[0] = 0;
+        hdr->sched[1] = 0;
+    }
     __syncthreads();
     bool bad = false;
     for (int64_t a = tid; a < TK; a += kPermThreads) {
         const int e = ids[a];
-        if (e < 0 || e >= kExperts) {
+        if (e < 0 || e >= n_valid) {
             bad = true;
             continue;
         }
@@ -60,6 +64,15 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
         hdr->tile_start[kExperts] = s / kRowPad;
         for (int e = nt; e < kExperts; ++e) hdr->touched[e] = -1;
         hdr->n_touched = nt;
+        int nf = 0, nm = 0;
+        for (int e = 0; e < kExperts; ++e) {
+            if (hist[e] > kFewTokens) hdr->many[nm++] = e;
+            else if (hist[e] > 0) hdr->few[nf++] = e;
+        }
+        for (int e = nf; e < kExperts; ++e) hdr->few[e] = -1;
+        for (int e = nm; e < kExperts; ++e) hdr->many[e] = -1;
+        hdr->n_few = nf;
+        hdr->n_many = nm;
     }
     __syncthreads();
     const unsigned lt_mask = (1u << lane) - 1u;
@@ -68,7 +81,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
         int e = -1;
         if (a < TK) {
             e = ids[a];
-            if (e < 0 || e >= kExperts) e = -1;
+            if (e < 0 || e >= n_valid) e = -1;
         }
         if (tid < kPermThreads / 32 * kExperts) wcount[tid / kExperts][tid % kExperts] = 0;
         __syncthreads();
@@ -97,14 +110,14 @@ __global__ void __launch_bounds__(kPermThreads) permute_kernel(const int32_t* __
         for (int r = seg[e] + hist[e] + tid; r < seg[e + 1]; r += kPermThreads) perm[r] = -1;
 }
 
-// x_perm[r] = x[perm[r] / K] for real rows (with `swap`, elements 1 and 2 of every group of 4
+// x_perm[r] = x[perm[r] / k_div] for real rows (k_div = K: assignment a belongs to token a / K) (with `swap`, elements 1 and 2 of every group of 4
 // swapped: the k order of the int8 tensor-core path), zeros for padding rows; rows past the last
 // segment are left alone.  16-byte vector copies, one warp per row.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ perm,
                                                           const WsHeader* __restrict__ hdr, int64_t d,
                                                           int64_t cap_rows, uint16_t* __restrict__ x_perm,
-                                                          int swap) {
+                                                          int swap, int k_div) {
     const int lane = threadIdx.x & 31;
     pdl_wait();
     pdl_trigger();
@@ -118,7 +131,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
         } else {
             // with int8 weights, elements 1 and 2 of every group of 4 swapped: the k order of the
             // converted weight tiles
-            const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(a / kTopK) * d);
+            const uint4* src = reinterpret_cast<const uint4*>(x + (int64_t)(a / k_div) * d);
             for (int64_t c = lane; c < chunks; c += 32) {
                 const uint4 v = ld_nc_v4(src + c);
                 dst[c] = swap ? make_uint4(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.x, v.y, 0x7632),
@@ -140,15 +153,23 @@ __global__ void __launch_bounds__(256) dense_setup_kernel(int64_t T, WsHeader* _
     const int64_t R = (T + kRowPad - 1) / kRowPad * kRowPad;
     if (blockIdx.x == 0 && threadIdx.x < kExperts) {
         const int e = threadIdx.x;
-        if (e == 0) hdr->status = 0;  // first kernel of a forward call to touch the header
+        if (e == 0) {  // first kernel of a forward call to touch the header
+            hdr->status = 0;
+            hdr->sched[0] = 0;
+            hdr->sched[1] = 0;
+        }
         hdr->counts[e] = (e == 0) ? (int32_t)T : 0;
         hdr->seg_start[e] = (e == 0) ? 0 : (int32_t)R;
         hdr->tile_start[e] = (e == 0) ? 0 : (int32_t)(R / kRowPad);
         hdr->touched[e] = (e == 0) ? 0 : -1;
+        hdr->few[e] = (e == 0 && T <= kFewTokens) ? 0 : -1;
+        hdr->many[e] = (e == 0 && T > kFewTokens) ? 0 : -1;
         if (e == 0) {
             hdr->seg_start[kExperts] = (int32_t)R;
             hdr->tile_start[kExperts] = (int32_t)(R / kRowPad);
             hdr->n_touched = 1;
+            hdr->n_few = (T <= kFewTokens) ? 1 : 0;
+            hdr->n_many = (T > kFewTokens) ? 1 : 0;
         }
     }
     for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < R; r += (int64_t)gridDim.x * blockDim.x) {
@@ -166,16 +187,23 @@ cudaError_t launch_dense_setup(int64_t T, WsHeader* hdr, int32_t* perm, float* w
 
 cudaError_t launch_permute(const int32_t* ids, int64_t T, WsHeader* hdr, int32_t* perm, int32_t* inv,
                            cudaStream_t st) {
-    return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), 0, st, ids, T * kTopK, hdr, perm, inv);
+    return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), 0, st, ids, T * kTopK, hdr, perm, inv, kExperts);
+}
+
+// The same over TK routing ids of any layout (one id per row: the rows an expert-parallel rank
+// received) naming experts 0 .. n_valid-1; other ids are skipped and reported (JMOE_DEV_BAD_INDEX).
+cudaError_t launch_permute_tk(const int32_t* ids, int64_t TK, int n_valid, WsHeader* hdr, int32_t* perm, int32_t* inv,
+                              cudaStream_t st) {
+    return launch_pdl(permute_kernel, dim3(1), dim3(kPermThreads), 0, st, ids, TK, hdr, perm, inv, n_valid);
 }
 
 cudaError_t launch_gather(const uint16_t* x, const int32_t* perm, const WsHeader* hdr, int64_t d, int64_t cap_rows,
-                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid) {
+                          uint16_t* x_perm, cudaStream_t st, int num_sms, bool swap_mid, int k_div) {
     int64_t blocks = (cap_rows + 7) / 8;
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     if (blocks < 1) blocks = 1;
     return launch_pdl(gather_rows_kernel, dim3((unsigned)blocks), dim3(256), 0, st, x, perm, hdr, d, cap_rows,
-                      x_perm, swap_mid ? 1 : 0);
+                      x_perm, swap_mid ? 1 : 0, k_div);
 }
 
 }  // namespace jmoe

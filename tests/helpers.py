@@ -19,12 +19,13 @@ def workload(name: str, **over) -> synth.Workload:
     return dataclasses.replace(wl, **over) if over else wl
 
 
-def gap_inputs(wl: synth.Workload, gap: float = GAP, max_rounds: int = 64):
+def gap_inputs(wl: synth.Workload, gap: float = GAP, max_rounds: int = 64, router_wl: Optional[synth.Workload] = None):
     """x, router weight and bias, with every row of x redrawn (next attempt number of its own
     stream) until its 2nd-vs-3rd router logit gap in fp64 exceeds `gap`, so that the top-2 set is
-    decided by the data and not by rounding.  Returns dict(x, wr, bias, attempts, redrawn)."""
-    wr = synth.gen_router(wl)
-    bias = synth.gen_bias(wl)
+    decided by the data and not by rounding.  The router comes from `router_wl` if given (ranks
+    that share one router but draw their own tokens).  Returns dict(x, wr, bias, attempts, redrawn)."""
+    wr = synth.gen_router(router_wl or wl)
+    bias = synth.gen_bias(router_wl or wl)
     attempts = np.zeros(wl.T, dtype=np.int64)
     x = synth.gen_x(wl)
     rows = np.arange(wl.T)

@@ -49,8 +49,8 @@ def test_tiny_all_tokens(tiny, path):
 
 
 @pytest.mark.parametrize("path", PATHS)
-@pytest.mark.parametrize("T,d,F", [(1, 256, 512), (3, 256, 512), (17, 384, 640), (129, 256, 512),
-                                   (300, 128, 128), (257, 512, 1152)])
+@pytest.mark.parametrize("T,d,F", [(1, 256, 512), (3, 256, 512), (17, 384, 640), (80, 384, 640), (96, 256, 512),
+                                   (129, 256, 512), (300, 128, 128), (257, 512, 1152)])
 def test_ragged_shapes(T, d, F, path):
     wl = dataclasses.replace(workload("tiny"), T=T, d=d, F=F)
     check_layer(Layer(wl), path)
