@@ -103,8 +103,8 @@ def algorithmic(kind, wl, T, touched, rows_padded, wbytes=1):
 
 
 def kernel_source_hash(kind):
-    files = {"gemv13": ["gemv.cu"], "gemv2": ["gemv.cu"], "gemm13": ["gemm_tc.cu", "tc.cuh"],
-             "gemm2": ["gemm_tc.cu", "tc.cuh"],
+    files = {"gemv13": ["gemv.cu"], "gemv2": ["gemv.cu"], "gemm13": ["gemm_ts.cu", "tc.cuh"],
+             "gemm2": ["gemm_ts.cu", "tc.cuh"],
              "quantize": ["quantize.cu"], "router": ["router.cu"], "combine": ["combine.cu"],
              "permute": ["permute.cu"], "gather": ["permute.cu"]}.get(kind, [])
     # the code only: comments are stripped and whitespace collapsed, so an edit of a comment keeps a

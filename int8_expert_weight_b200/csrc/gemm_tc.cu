@@ -1,30 +1,29 @@
-// Prefill path of the expert FFN: grouped GEMMs on the 5th-generation tensor cores (tcgen05), with
-// the ExpertsInt8 dequantization inside the kernel (Jamba-1.5 paper, §3.1: int8 weight tiles move
-// HBM -> SRAM and are turned into BF16 there, right before the matrix math).
+// Prefill path of the two comparator layers: grouped GEMMs on the 5th-generation tensor cores
+// (tcgen05) for unquantized bf16 weights and for FP8 (E4M3) weights and activations, the layers
+// the Jamba-1.5 paper measures ExpertsInt8 against (§3.1).  The ExpertsInt8 GEMMs themselves are
+// in gemm_ts.cu.
 //
-//   gemm13: h[r][j] = bf16( SiLU(S1[j] * (x_r . Q1[j])) * (S3[j] * (x_r . Q3[j])) )   tile: 128 rows x
-//           (128 j of Q1 | the same 128 j of Q3), so both halves of SwiGLU meet in one accumulator
-//   gemm2:  out[a][i] = p_a * S2[i] * (h_r . Q2[i])                                   tile: 128 rows x BN i
+//   gemm13: h[r][j] = bf16( SiLU(g_r . W1[j]) * (u_r . W3[j]) )     tile: 128 rows x (128 j of W1 |
+//           the same 128 j of W3), so both halves of SwiGLU meet in one accumulator
+//   gemm2:  out[a][i] = p_a * (h_r . W2[i])                         tile: 128 rows x BN i
 //
-// Persistent: one CTA per SM walks the tile list with stride gridDim.x; 448 threads in roles:
-//   warp 0       TMA producer: activation tile (bf16, SWIZZLE_128B) + int8 weight tile per 64-wide K step
-//   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128, N=BN, K=16, fp32 in TMEM
-//   warps 2-9    converters: int8 tile -> bf16 in the canonical SWIZZLE_128B K-major layout
-//   warps 10-13  epilogue: tcgen05.ld, scales, SiLU * up or routing weight, global stores
-// A 3-stage ring of (activations, int8 weights, bf16 weights) buffers with full / converted / empty
-// mbarriers, and two TMEM accumulators (full / empty mbarriers) so that a tile's epilogue overlaps
-// the next tile's main loop.  Every wait is bounded: on timeout the kernel records
-// JMOE_DEV_TIMEOUT in the workspace status word, the other roles stop at their next wait,
-// outstanding copies and MMAs are waited for (bounded), TMEM is released and the CTA returns.
+// Persistent: one CTA per SM walks the tile list with stride gridDim.x; 192 threads in roles:
+//   warp 0       TMA producer: activation tile + weight tile per K step, both straight into the
+//                MMA's SWIZZLE_128B K-major layout (128 bytes of K per row)
+//   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16 (bf16) or kind::f8f6f4 (E4M3),
+//                M=128, N=BN, fp32 accumulators in TMEM
+//   warps 2-5    epilogue: tcgen05.ld, scales, SiLU * up or routing weight, global stores
+// A 4-stage ring of (activation, weight) buffers with full / empty mbarriers, and two TMEM
+// accumulators (full / empty mbarriers) so that a tile's epilogue overlaps the next tile's main
+// loop.  Every wait is bounded: on timeout the kernel records JMOE_DEV_TIMEOUT in the workspace
+// status word, the other roles stop at their next wait, outstanding copies and MMAs are waited
+// for (bounded), TMEM is released and the CTA returns.
 //
 // Tiles are ordered expert by expert; inside an expert, bands of M tiles keep their activations
 // resident in L2 while every N tile of the weights streams past once per band.
 //
-// The same kernel serves three weight formats (template flags): int8 codes (kW8, the layer above),
-// unquantized bf16 weights (TMA straight into the MMA's tile, 4 stages, converters idle), and the
-// FP8 comparator (kF8: E4M3 activations and weights, both by TMA, 128 K elements per stage,
-// kind::f8f6f4 MMAs, per-row activation scales in the epilogue, bf16 h).  The W2 epilogue can also
-// write y in bf16 directly (the dense MLP, one assignment per token) instead of fp32 slots.
+// FP8 (kF8): E4M3 activations and weights, 128 K elements per stage, kind::f8f6f4 MMAs, per-row
+// activation scales and per-channel weight scales in the epilogue, bf16 h.
 #include <cuda.h>
 
 #include <atomic>
@@ -36,17 +35,15 @@ namespace jmoe {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kConvWarps = 8;
 constexpr int kEpiWarps = 4;
-constexpr int kGemmThreads = (2 + kConvWarps + kEpiWarps) * 32;
+constexpr int kGemmThreads = (2 + kEpiWarps) * 32;
 constexpr uint32_t kMaxPolls = 1u << 22;       // ~0.3 s of polling: far above any healthy wait
-constexpr uint32_t kTestMaxPolls = 1u << 14;   // short bound used together with the test hook
 
 struct GemmArgs {
     WsHeader* hdr;
     const int32_t* perm;  // assignment index of each permuted row, -1 = padding
-    const float* sa;      // gemm13: S1 [E][N]; gemm2: S2 [E][N]
-    const float* sb;      // gemm13: S3 [E][N]
+    const float* sa;      // FP8 gemm13: S1 [E][N]; FP8 gemm2: S2 [E][N]
+    const float* sb;      // FP8 gemm13: S3 [E][N]
     const float* wts;     // gemm2: routing weight per assignment
     uint16_t* h_out;      // gemm13: h [rows][N]
     float* slot_out;      // gemm2: out_slot [T*K][N]
@@ -55,43 +52,21 @@ struct GemmArgs {
     int n_tiles;          // N tiles per M tile
     int band;             // M tiles per raster band
     uint32_t max_polls;   // bound of every mbarrier wait
-    int skip_copy;        // test hook: CTA 0 skips the copies of its second K step (a wait then runs out)
-    uint16_t* y_out;      // gemm2 of the dense MLP: y [T][N] in bf16, written instead of out_slot
     // FP8 layer only: per-row activation scale (gemm13: per token, indexed by assignment / K;
     // gemm2: per permuted row)
     const float* a_scale;
 };
 
-// Shared-memory ring: per stage the activation tile, the bf16 weight tile the MMA reads and, for
-// int8 weights, the int8 tile as loaded (converted into the bf16 tile by the converter warps).
-// Unquantized bf16 weights are loaded straight into the bf16 tile, which leaves room for 4 stages.
-template <int BN, bool kW8>
+// Shared-memory ring: per stage the activation tile and the weight tile, both as the MMA reads
+// them (128 bytes of K per row: 64 bf16 or 128 E4M3).
+template <int BN>
 struct StageLayout {
-    static constexpr int kStages = kW8 ? 3 : 4;
-    static constexpr int kA = kBM * kBK * 2;          // bf16 activations
-    static constexpr int kBbf = BN * kBK * 2;         // bf16 weights (converted or loaded)
-    static constexpr int kBq = kW8 ? BN * kBK : 0;    // int8 weights (as loaded)
-    static constexpr int kStage = kA + kBbf + kBq;
+    static constexpr int kStages = 4;
+    static constexpr int kA = kBM * 128;              // activations
+    static constexpr int kB = BN * 128;               // weights
+    static constexpr int kStage = kA + kB;
     static constexpr int kSmem = kStages * kStage + 1024 + 256;
 };
-
-// 16 int8 weights -> 8 bf16x2 words, exactly.  Word i of the input (bytes b0..b3) yields the pairs
-// (b0, b2) and (b1, b3), so within every group of 4 the stored k order is 0, 2, 1, 3; the
-// activation operands of this path are stored with the same order (elements 1 and 2 of each group
-// of 4 swapped), and a k-permutation applied to both operands leaves every dot product unchanged.
-__device__ __forceinline__ void convert16(const uint4 v, uint32_t (&o)[8], const S8Consts& k) {
-    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o[2 * i] = s8x2_even_to_bf16x2(w[i], k);
-        o[2 * i + 1] = s8x2_odd_to_bf16x2(w[i], k);
-    }
-}
-
-// Swap elements 1 and 2 of a group of 4 bf16 held as two bf16x2 words (lo = e0 e1, hi = e2 e3).
-__device__ __forceinline__ uint2 swap_mid4(uint32_t lo, uint32_t hi) {
-    return make_uint2(__byte_perm(lo, hi, 0x5410), __byte_perm(lo, hi, 0x7632));
-}
 
 __device__ __forceinline__ void fail(WsHeader* hdr, volatile int* abort) {
     *abort = 1;
@@ -126,11 +101,11 @@ __device__ __forceinline__ bool tile_coord(const WsHeader* hdr, const GemmArgs& 
 
 // kF8: both operands E4M3 codes copied by TMA into the MMA's layout (no conversion), 128 K
 // elements (128 bytes) per stage, kind::f8f6f4 MMAs, activation and weight scales in the epilogue.
-template <bool kDual, int BN, bool kW8, bool kF8 = false>
+template <bool kDual, int BN, bool kF8>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmB1, GemmArgs p) {
-    using SL = StageLayout<BN, kW8>;
+    using SL = StageLayout<BN>;
     constexpr int kStages = SL::kStages;
     static_assert(!kDual || BN == 256, "the SwiGLU tile pairs 128 gate rows with 128 up rows");
     constexpr uint32_t kTmemCols = 2 * BN;  // two accumulators
@@ -146,20 +121,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kStages * SL::kStage);
     uint64_t* full_tma = bars;                  // [kStages] TMA bytes landed
-    uint64_t* full_bf = bars + kStages;         // [kStages] converted by all converter warps
-    uint64_t* empty = bars + 2 * kStages;       // [kStages] MMAs reading the stage are done
-    uint64_t* acc_full = bars + 3 * kStages;    // [2] accumulator complete
+    uint64_t* empty = bars + kStages;           // [kStages] MMAs reading the stage are done
+    uint64_t* acc_full = bars + 2 * kStages;    // [2] accumulator complete
     uint64_t* acc_empty = acc_full + 2;         // [2] accumulator read out by the epilogue
     uint64_t* mma_done = acc_empty + 2;         // every issued MMA complete (teardown)
     auto sA = [&](int s) { return smem + s * SL::kStage; };
-    auto sBbf = [&](int s) { return smem + s * SL::kStage + SL::kA; };
-    auto sBq = [&](int s) { return smem + s * SL::kStage + SL::kA + SL::kBbf; };
+    auto sB = [&](int s) { return smem + s * SL::kStage + SL::kA; };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
             tc::mbar_init(&full_tma[s], 1);
-            tc::mbar_init(&full_bf[s], kConvWarps);
             tc::mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -180,10 +152,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_holder;
-    static_assert(!(kW8 && kF8), "one weight format");
     constexpr int kKStage = kF8 ? 128 : kBK;  // K elements per stage (128 bytes per row either way)
     const int KB = p.K / kKStage;
-    constexpr uint32_t kTxBytes = SL::kA + (kW8 ? SL::kBq : SL::kBbf);
+    constexpr uint32_t kTxBytes = SL::kA + SL::kB;
     constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, BN);
     constexpr uint32_t kIdescF8 = tc::idesc_e4m3_f32(kBM, BN);
     int issued_round[kStages];  // producer: last round issued on each stage (-1: none)
@@ -208,18 +179,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         ok = false;
                         break;
                     }
-                    if (p.skip_copy && blockIdx.x == 0 && L == (int)blockIdx.x && kb == 1) continue;
                     tc::mbar_arrive_expect_tx(&full_tma[s], kTxBytes);
                     tc::tma_load_2d(sA(s), &tmA, &full_tma[s], kb * kKStage, a_row0);
-                    if (kW8) {
-                        tc::tma_load_2d(sBq(s), &tmB0, &full_tma[s], kb * kBK, w_row0);
-                        if (kDual)
-                            tc::tma_load_2d(sBq(s) + (BN / 2) * kBK, &tmB1, &full_tma[s], kb * kBK, w_row0);
-                    } else {  // bf16 weights land in the MMA's SWIZZLE_128B tile directly (128 bytes per row)
-                        tc::tma_load_2d(sBbf(s), &tmB0, &full_tma[s], kb * kKStage, w_row0);
-                        if (kDual)
-                            tc::tma_load_2d(sBbf(s) + (BN / 2) * 128, &tmB1, &full_tma[s], kb * kKStage, w_row0);
-                    }
+                    tc::tma_load_2d(sB(s), &tmB0, &full_tma[s], kb * kKStage, w_row0);
+                    if (kDual) tc::tma_load_2d(sB(s) + (BN / 2) * 128, &tmB1, &full_tma[s], kb * kKStage, w_row0);
                     issued_round[s] = r;
                 }
                 if (!ok) break;
@@ -240,15 +203,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int s = g % kStages, r = g / kStages;
-                    if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls) ||
-                        (kW8 && !tc::mbar_wait_bounded(&full_bf[s], r & 1, &abort_flag, p.max_polls))) {
+                    if (!tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls)) {
                         if (!abort_flag) fail(p.hdr, &abort_flag);
                         ok = false;
                         break;
                     }
                     tc::tc_fence_after();
                     const uint64_t adesc = tc::sw128_kmajor_desc(tc::smem_u32(sA(s)));
-                    const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sBbf(s)));
+                    const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sB(s)));
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {  // +32 bytes per K step (16 bf16 or 32 fp8) = +2 in the address field
                         if (kF8)
@@ -265,44 +227,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc::mma_commit(mma_done);  // arrives once every MMA issued above has completed
         }
         __syncwarp();
-    } else if (warp < 2 + kConvWarps) {
-        if (kW8) {  // bf16 weights need no conversion
-        // ---------------- converters: int8 tile -> bf16, canonical SWIZZLE_128B K-major (16-byte
-        // chunk c of row r stored at chunk c ^ (r & 7) of the row's 128 bytes)
-        const int t = threadIdx.x - 64;
-        const S8Consts k8 = s8_consts();
-        int g = 0;
-        for (int L = blockIdx.x; L < total; L += gridDim.x) {
-            if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
-            bool ok = true;
-            for (int kb = 0; kb < KB; ++kb, ++g) {
-                const int s = g % kStages, r = g / kStages;
-                const bool landed = tc::mbar_wait_bounded(&full_tma[s], r & 1, &abort_flag, p.max_polls);
-                if (!__all_sync(0xffffffffu, landed)) {  // warp-uniform: __syncwarp below needs all lanes
-                    if (!abort_flag) fail(p.hdr, &abort_flag);
-                    ok = false;
-                    break;
-                }
-                const uint8_t* q8 = sBq(s);
-                uint8_t* bf = sBbf(s);
-#pragma unroll
-                for (int i = 0; i < BN * 4 / (kConvWarps * 32); ++i) {
-                    const int qi = t + kConvWarps * 32 * i, row = qi >> 2, c = qi & 3;
-                    const uint4 v = *reinterpret_cast<const uint4*>(q8 + row * kBK + c * 16);
-                    uint32_t o[8];
-                    convert16(v, o, k8);
-                    uint8_t* rp = bf + row * 128;
-                    *reinterpret_cast<uint4*>(rp + (((2 * c) ^ (row & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-                    *reinterpret_cast<uint4*>(rp + (((2 * c + 1) ^ (row & 7)) << 4)) =
-                        make_uint4(o[4], o[5], o[6], o[7]);
-                }
-                tc::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&full_bf[s]);
-            }
-            if (!ok) break;
-        }
-        }
     } else {
         // ---------------- epilogue
         const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
@@ -363,60 +287,24 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tc::tmem_wait_ld();
                     uint32_t packed[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const float g0 = __uint_as_float(a1[i]) * (kW8 ? __ldg(s1 + c + i) : 1.0f);
-                        const float g1 = __uint_as_float(a1[i + 1]) * (kW8 ? __ldg(s1 + c + i + 1) : 1.0f);
-                        const float u0 = __uint_as_float(a3[i]) * (kW8 ? __ldg(s3 + c + i) : 1.0f);
-                        const float u1 = __uint_as_float(a3[i + 1]) * (kW8 ? __ldg(s3 + c + i + 1) : 1.0f);
+                    for (int i = 0; i < 32; i += 2) {  // bf16 weights: no scales
+                        const float g0 = __uint_as_float(a1[i]), g1 = __uint_as_float(a1[i + 1]);
+                        const float u0 = __uint_as_float(a3[i]), u1 = __uint_as_float(a3[i + 1]);
                         packed[i / 2] = (uint32_t)f32_to_bf16_bits(silu(g0) * u0) |
                                         ((uint32_t)f32_to_bf16_bits(silu(g1) * u1) << 16);
                     }
-                    // h feeds the down-projection GEMM as its activation operand: with int8 weights,
-                    // store every group of 4 columns in the 0, 2, 1, 3 order the weight conversion produces
                     uint4* dst = reinterpret_cast<uint4*>(hrow + c);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (kW8) {
-                            const uint2 a = swap_mid4(packed[4 * v], packed[4 * v + 1]);
-                            const uint2 b = swap_mid4(packed[4 * v + 2], packed[4 * v + 3]);
-                            dst[v] = make_uint4(a.x, a.y, b.x, b.y);
-                        } else {
-                            dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
-                        }
-                    }
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
                 }
             } else {
                 const int i0 = t.n_tile * BN;
                 const int32_t a = p.perm[gr];
                 // FP8: the routing weight times the row's activation (h) scale
                 const float wt = a >= 0 ? p.wts[a] * (kF8 ? p.a_scale[gr] : 1.0f) : 0.0f;
-                const float* s2 = p.sa + (int64_t)t.e * p.N + i0;
-                if (p.y_out) {
-                    // dense MLP: one assignment per token, its output rounded to bf16 here
-                    uint16_t* yrow = p.y_out + (int64_t)(a >= 0 ? a / kTopK : 0) * p.N + i0;
-#pragma unroll 1
-                    for (int c = 0; c < BN; c += 32) {
-                        uint32_t v[32];
-                        tc::tmem_ld32(tbase + c, v);
-                        tc::tmem_wait_ld();
-                        if (a >= 0) {
-                            uint32_t packed[16];
-#pragma unroll
-                            for (int i = 0; i < 32; i += 2) {
-                                const float o0 = wt * ((kW8 || kF8 ? __ldg(s2 + c + i) : 1.0f) * __uint_as_float(v[i]));
-                                const float o1 =
-                                    wt * ((kW8 || kF8 ? __ldg(s2 + c + i + 1) : 1.0f) * __uint_as_float(v[i + 1]));
-                                packed[i / 2] =
-                                    (uint32_t)f32_to_bf16_bits(o0) | ((uint32_t)f32_to_bf16_bits(o1) << 16);
-                            }
-                            uint4* dst = reinterpret_cast<uint4*>(yrow + c);
-#pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2],
-                                                    packed[4 * k + 3]);
-                        }
-                    }
-                } else {
+                const float* s2 = kF8 ? p.sa + (int64_t)t.e * p.N + i0 : nullptr;
+                {
                     float* orow = p.slot_out + (int64_t)(a >= 0 ? a : 0) * p.N + i0;
 #pragma unroll 1
                     for (int c = 0; c < BN; c += 32) {
@@ -428,10 +316,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
                                 float4 o;
-                                o.x = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
-                                o.y = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
-                                o.z = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
-                                o.w = wt * ((kW8 || kF8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
+                                o.x = wt * ((kF8 ? __ldg(s2 + c + 4 * k + 0) : 1.0f) * __uint_as_float(v[4 * k + 0]));
+                                o.y = wt * ((kF8 ? __ldg(s2 + c + 4 * k + 1) : 1.0f) * __uint_as_float(v[4 * k + 1]));
+                                o.z = wt * ((kF8 ? __ldg(s2 + c + 4 * k + 2) : 1.0f) * __uint_as_float(v[4 * k + 2]));
+                                o.w = wt * ((kF8 ? __ldg(s2 + c + 4 * k + 3) : 1.0f) * __uint_as_float(v[4 * k + 3]));
                                 dst[k] = o;
                             }
                         }
@@ -501,18 +389,18 @@ bool make_map(CUtensorMap* m, const void* ptr, CUtensorMapDataType dt, int elem_
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int band_for(int K) {
-    // keep a band's activation tiles (band * 128 rows * K * 2 bytes) near 24 MB of L2
-    const int64_t per_tile = (int64_t)kBM * K * 2;
+int band_for(int K, int act_bytes) {
+    // keep a band's activation tiles (band * 128 rows * K elements) near 24 MB of L2
+    const int64_t per_tile = (int64_t)kBM * K * act_bytes;
     int b = (int)((24ll << 20) / per_tile);
     return b < 1 ? 1 : (b > 16 ? 16 : b);
 }
 
-template <bool kDual, int BN, bool kW8, bool kF8 = false>
+template <bool kDual, int BN, bool kF8>
 cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const CUtensorMap& tb1, const GemmArgs& p,
                           int64_t m_tiles_cap, cudaStream_t st) {
-    using SL = StageLayout<BN, kW8>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN, kW8, kF8>,
+    using SL = StageLayout<BN>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<kDual, BN, kF8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, SL::kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (fewer when there are fewer tile slots)
@@ -526,7 +414,7 @@ cudaError_t launch_gemm_t(const CUtensorMap& ta, const CUtensorMap& tb0, const C
     }
     int64_t grid = m_tiles_cap * p.n_tiles;
     if (grid > sms) grid = sms;
-    return launch_pdl(gemm_tc_kernel<kDual, BN, kW8, kF8>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta,
+    return launch_pdl(gemm_tc_kernel<kDual, BN, kF8>, dim3((unsigned)grid), dim3(kGemmThreads), SL::kSmem, st, ta,
                       tb0, tb1, p);
 }
 
@@ -547,8 +435,8 @@ cudaError_t launch_gemm13_bf16w(WsHeader* hdr, const int32_t* perm, const uint16
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,          perm,          nullptr,     nullptr,
                nullptr,      h,             nullptr,     (int)d,
-               (int)F,       (int)(F / 128), band_for((int)d), kMaxPolls,
-               0};
+               (int)F,       (int)(F / 128), band_for((int)d, 2), kMaxPolls,
+               nullptr};
     return launch_gemm_t<true, 256, false>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
@@ -563,8 +451,8 @@ cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,         perm,         nullptr,     nullptr,
                wts,         nullptr,      out_slot,    (int)F,
-               (int)d,      (int)(d / BN), band_for((int)F), kMaxPolls,
-               0};
+               (int)d,      (int)(d / BN), band_for((int)F, 2), kMaxPolls,
+               nullptr};
     if (BN == 256) return launch_gemm_t<false, 256, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
@@ -583,9 +471,9 @@ cudaError_t launch_gemm13_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* 
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,          perm,          S1,          S3,
                nullptr,      h,             nullptr,     (int)d,
-               (int)F,       (int)(F / 128), band_for((int)d), kMaxPolls,
-               0,            nullptr,       sx};
-    return launch_gemm_t<true, 256, false, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
+               (int)F,       (int)(F / 128), band_for((int)d, 1), kMaxPolls,
+               sx};
+    return launch_gemm_t<true, 256, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
 // out_slot[a] = p_a * sh_r * S2 . (h8_r . Q2^T): E4M3 h8 [rows_cap][F] with per-row scales sh.
@@ -600,10 +488,10 @@ cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h
         return cudaErrorInvalidValue;
     GemmArgs p{hdr,         perm,         S2,          nullptr,
                wts,         nullptr,      out_slot,    (int)F,
-               (int)d,      (int)(d / BN), band_for((int)F), kMaxPolls,
-               0,           nullptr,      sh};
-    if (BN == 256) return launch_gemm_t<false, 256, false, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
-    return launch_gemm_t<false, 128, false, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
+               (int)d,      (int)(d / BN), band_for((int)F, 1), kMaxPolls,
+               sh};
+    if (BN == 256) return launch_gemm_t<false, 256, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
+    return launch_gemm_t<false, 128, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
 
 }  // namespace jmoe

@@ -54,16 +54,18 @@ namespace jmoe {
 namespace ts {
 
 constexpr int kWRows = 128;   // weight rows per tile (MMA M, TMEM lanes)
-constexpr int kTokMax = 192;  // tokens per tile at most (MMA N)
-constexpr int kAccBufs = 2;   // TMEM accumulators: the epilogue of one tile overlaps the next tile's MMAs
+constexpr int kTokMax = 256;  // tokens per tile at most (MMA N)
+constexpr int kAccBufs = 1;   // TMEM accumulators (one of 256 columns leaves 256 for the weight ring)
 constexpr int kBK = 64;       // K elements per pipeline step
-constexpr int kXStages = 7;
+constexpr int kXStages = 5;
 constexpr int kQStages = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
 constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
 constexpr int kTileSlots = 4;
-constexpr int kConvWarps = 8;
+constexpr int kConvWarps = 16;                 // four per TMEM lane quarter
+constexpr int kConvK = kBK / (kConvWarps / 4);  // K elements of a step each converter warp takes
+static_assert(kConvK == 16 || kConvK == 32, "converter split");
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kConvWarps + kEpiWarps) * 32;
 constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
@@ -136,6 +138,10 @@ __device__ __forceinline__ bool tile_at(const WsHeader* hdr, const Args& p, int 
     }
     return false;
 }
+
+// tcgen05.st of a converter's bf16 pairs: 8 or 16 columns.
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t (&r)[8]) { tc::tmem_st8(taddr, r); }
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t (&r)[16]) { tc::tmem_st16(taddr, r); }
 
 // SiLU with the fast exponential and division intrinsics: a few fp32 ulps from the exact value,
 // far below the bf16 rounding of h that follows.
@@ -334,13 +340,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 2 + kConvWarps) {
         // ---------------- converters: int8 [128][64] (SWIZZLE_64B: 16-byte chunk c of row r at
         // chunk c ^ ((r >> 1) & 3)) -> bf16 pairs in TMEM lane = tile row
-        const int cw = warp - 2, qd = warp & 3, khalf = cw >> 2;
+        constexpr int kChunks = kConvK / 16;  // 16-byte chunks of its row a converter takes per step
+        const int cw = warp - 2, qd = warp & 3, kpart = cw >> 2;
         const int trow = 32 * qd + lane;  // TMEM lane = tile row this thread converts
         const int srow = kDual ? ((lane < 16) ? 16 * qd + lane : kWRows / 2 + 16 * qd + lane - 16) : trow;
         const int sw = (srow >> 1) & 3;
-        const uint32_t c0 = (uint32_t)(srow * 64 + (((2 * khalf) ^ sw) << 4));
-        const uint32_t c1 = (uint32_t)(srow * 64 + (((2 * khalf + 1) ^ sw) << 4));
-        const uint32_t t_lane = tmem + ((uint32_t)(32 * qd) << 16) + kACol0 + (uint32_t)(16 * khalf);
+        uint32_t coff[kChunks];
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) coff[i] = (uint32_t)(srow * 64 + (((kpart * kChunks + i) ^ sw) << 4));
+        const uint32_t t_lane =
+            tmem + ((uint32_t)(32 * qd) << 16) + kACol0 + (uint32_t)(kpart * (kConvK / 2));
         const S8Consts k8 = s8_consts();
         int g = 0;
         for (int it = 0;; ++it) {
@@ -359,16 +368,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint8_t* q8 = sQ + sq * kQBytes;
-                const uint4 v0 = *reinterpret_cast<const uint4*>(q8 + c0);
-                const uint4 v1 = *reinterpret_cast<const uint4*>(q8 + c1);
+                uint4 v[kChunks];
+#pragma unroll
+                for (int i = 0; i < kChunks; ++i) v[i] = *reinterpret_cast<const uint4*>(q8 + coff[i]);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&q_empty[sq]);
-                uint32_t o[16];
-                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                uint32_t o[kConvK / 2];
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    o[2 * i] = s8x2_even_to_bf16x2(w[i], k8);
-                    o[2 * i + 1] = s8x2_odd_to_bf16x2(w[i], k8);
+                for (int i = 0; i < kChunks; ++i) {
+                    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        o[8 * i + 2 * j] = s8x2_even_to_bf16x2(w[j], k8);
+                        o[8 * i + 2 * j + 1] = s8x2_odd_to_bf16x2(w[j], k8);
+                    }
                 }
                 bool free_ = ra == 0 || tc::mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1, &abort_flag, p.max_polls);
                 if (!__all_sync(0xffffffffu, free_)) {
@@ -377,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc::tc_fence_after();
-                tc::tmem_st16(t_lane + (uint32_t)(sa * 32), o);
+                tmem_st_n(t_lane + (uint32_t)(sa * 32), o);
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();

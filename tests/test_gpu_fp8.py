@@ -19,8 +19,8 @@ import int8_expert_weight_b200 as jm  # noqa: E402
 import oracle  # noqa: E402
 import synth  # noqa: E402
 from gpu_layer import bf16_to_dev, dev_to_bf16_bits  # noqa: E402
-from helpers import (assert_routing, assert_y_close, gap_inputs, tile_covering_tokens,  # noqa: E402
-                     uncovered_tiles, workload)
+from helpers import (Y_ABS, Y_MEAN_REL, assert_routing, assert_y_close, gap_inputs,  # noqa: E402
+                     tile_covering_tokens, uncovered_tiles, workload, y_errors)
 from oracle_pins import E4M3_VALUES, bf16_bits  # noqa: E402
 
 PATHS = [pytest.param(jm.PATH_GEMV, id="gemv"), pytest.param(jm.PATH_GEMM, id="gemm")]
@@ -90,18 +90,48 @@ class F8Layer:
         torch.cuda.synchronize()
         return dev_to_bf16_bits(y), ids.cpu().numpy(), w.cpu().numpy()
 
-    def ref(self, tokens=None):
+    def ref(self, tokens=None, want_hidden=False):
         return oracle.moe_forward_fp8(self.x_bits, self.wr, self.bias, self.q["w1"], self.s["w1"], self.q["w3"],
-                                      self.s["w3"], self.q["w2"], self.s["w2"], tokens=tokens)
+                                      self.s["w3"], self.q["w2"], self.s["w2"], tokens=tokens,
+                                      want_hidden=want_hidden)
+
+
+# The GPU's SwiGLU value before its bf16 rounding is within this relative distance of the exact
+# one: its dot products add exact E4M3 x E4M3 products in fp32, whose rounding errors grow like
+# sqrt(K) fp32 ulps (K <= 16384 here: 128 * 2^-24 = 2^-17), and SiLU and the product with the up
+# value add a few ulps more; twice that is allowed.  It is far below a bf16 step (2^-8).
+H_REL = 2.0 ** -16
+
+
+def scale_ambiguous(h: np.ndarray) -> np.ndarray:
+    """Per row of fp64 SwiGLU values h [..., F]: whether the row's E4M3 scale (its largest |bf16 h|
+    over 448) is not decided by the exact values, because the largest |h| lies within H_REL of a
+    bf16 rounding boundary, so that both neighbouring bf16 values are results a correct fp32
+    computation can round to; the row's codes then follow either scale."""
+    m = np.abs(h).max(-1)
+    lo = synth.f32_to_bf16_bits((m * (1 - H_REL)).astype(np.float32))
+    hi = synth.f32_to_bf16_bits((m * (1 + H_REL)).astype(np.float32))
+    return lo != hi
 
 
 def check(L, path, tokens=None):
+    """Routing exact; y within the layer tolerance on every token whose two SwiGLU rows have their
+    E4M3 scales decided, and within twice that on the rest (one bf16 step in a row's scale moves
+    its codes by at most one E4M3 step each); the mean relative error over all tokens as usual."""
     y, ids, w = L.forward(path)
-    ref = L.ref(tokens)
+    ref = L.ref(tokens, want_hidden=True)
     sel = slice(None) if tokens is None else np.asarray(tokens)
     _, _, z = oracle.route(L.x_bits[sel], L.wr, L.bias, want_logits=True)
     assert_routing(ids[sel], w[sel], ref["ids"], ref["w"], z)
-    return assert_y_close(y[sel], ref["y"])
+    amb = scale_ambiguous(ref["h"]).any(-1)
+    ys = y[sel]
+    if (~amb).any():
+        assert_y_close(ys[~amb], ref["y"][~amb], "y, tokens with decided scales")
+    if amb.any():
+        err, _ = y_errors(ys[amb], ref["y"][amb])
+        assert err <= 2 * Y_ABS, f"y, tokens with an undecided scale: {err:.3e}"
+    _, mean_rel = y_errors(ys, ref["y"])
+    assert mean_rel <= Y_MEAN_REL, f"mean relative error {mean_rel:.3e}"
 
 
 @pytest.mark.parametrize("path", PATHS)
