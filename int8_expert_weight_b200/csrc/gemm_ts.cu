@@ -63,9 +63,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
 constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
 constexpr int kTileSlots = 4;
-constexpr int kConvWarps = 16;                 // four per TMEM lane quarter
-constexpr int kConvK = kBK / (kConvWarps / 4);  // K elements of a step each converter warp takes
-static_assert(kConvK == 16 || kConvK == 32, "converter split");
+constexpr int kConvWarps = 16;               // four per TMEM lane quarter
+constexpr int kConvGroups = kConvWarps / 4;  // warps of a quarter take turns: stage g goes to group g % 4
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kConvWarps + kEpiWarps) * 32;
 constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
@@ -195,10 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < kQStages; ++s) {
             tc::mbar_init(&q_full[s], 1);
-            tc::mbar_init(&q_empty[s], kConvWarps);
+            tc::mbar_init(&q_empty[s], 4);
         }
         for (int s = 0; s < kAStages; ++s) {
-            tc::mbar_init(&a_full[s], kConvWarps);
+            tc::mbar_init(&a_full[s], 4);
             tc::mbar_init(&a_empty[s], 1);
         }
         for (int s = 0; s < kTileSlots; ++s) {
@@ -340,16 +339,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp < 2 + kConvWarps) {
         // ---------------- converters: int8 [128][64] (SWIZZLE_64B: 16-byte chunk c of row r at
         // chunk c ^ ((r >> 1) & 3)) -> bf16 pairs in TMEM lane = tile row
-        constexpr int kChunks = kConvK / 16;  // 16-byte chunks of its row a converter takes per step
-        const int cw = warp - 2, qd = warp & 3, kpart = cw >> 2;
+        const int cw = warp - 2, qd = warp & 3, grp = cw >> 2;
         const int trow = 32 * qd + lane;  // TMEM lane = tile row this thread converts
         const int srow = kDual ? ((lane < 16) ? 16 * qd + lane : kWRows / 2 + 16 * qd + lane - 16) : trow;
         const int sw = (srow >> 1) & 3;
-        uint32_t coff[kChunks];
+        uint32_t coff[4];
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) coff[i] = (uint32_t)(srow * 64 + (((kpart * kChunks + i) ^ sw) << 4));
-        const uint32_t t_lane =
-            tmem + ((uint32_t)(32 * qd) << 16) + kACol0 + (uint32_t)(kpart * (kConvK / 2));
+        for (int i = 0; i < 4; ++i) coff[i] = (uint32_t)(srow * 64 + ((i ^ sw) << 4));
+        const uint32_t t_lane = tmem + ((uint32_t)(32 * qd) << 16) + kACol0;
         const S8Consts k8 = s8_consts();
         int g = 0;
         for (int it = 0;; ++it) {
@@ -359,6 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, L >= 0)) break;  // warp-uniform
             bool ok = true;
             for (int kb = 0; kb < KB; ++kb, ++g) {
+                if (g % kConvGroups != grp) continue;  // another warp of this quarter takes this step
                 const int sq = g % kQStages, rq = g / kQStages;
                 const int sa = g % kAStages, ra = g / kAStages;
                 bool landed = tc::mbar_wait_bounded(&q_full[sq], rq & 1, &abort_flag, p.max_polls);
@@ -368,19 +366,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint8_t* q8 = sQ + sq * kQBytes;
-                uint4 v[kChunks];
+                uint4 v[4];
 #pragma unroll
-                for (int i = 0; i < kChunks; ++i) v[i] = *reinterpret_cast<const uint4*>(q8 + coff[i]);
+                for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(q8 + coff[i]);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&q_empty[sq]);
-                uint32_t o[kConvK / 2];
+                uint32_t o0[16], o1[16];
 #pragma unroll
-                for (int i = 0; i < kChunks; ++i) {
+                for (int i = 0; i < 4; ++i) {
                     const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        o[8 * i + 2 * j] = s8x2_even_to_bf16x2(w[j], k8);
-                        o[8 * i + 2 * j + 1] = s8x2_odd_to_bf16x2(w[j], k8);
+                        uint32_t* o = (i < 2) ? o0 : o1;
+                        o[8 * (i & 1) + 2 * j] = s8x2_even_to_bf16x2(w[j], k8);
+                        o[8 * (i & 1) + 2 * j + 1] = s8x2_odd_to_bf16x2(w[j], k8);
                     }
                 }
                 bool free_ = ra == 0 || tc::mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1, &abort_flag, p.max_polls);
@@ -390,7 +389,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc::tc_fence_after();
-                tmem_st_n(t_lane + (uint32_t)(sa * 32), o);
+                tc::tmem_st16(t_lane + (uint32_t)(sa * 32), o0);
+                tc::tmem_st16(t_lane + (uint32_t)(sa * 32 + 16), o1);
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
