@@ -58,7 +58,7 @@ constexpr int kTokMax = 256;  // tokens per tile at most (MMA N)
 constexpr int kAccBufs = 1;   // TMEM accumulators (one of 256 columns leaves 256 for the weight ring)
 constexpr int kBK = 64;       // K elements per pipeline step
 constexpr int kXStages = 5;
-constexpr int kQStages = 6;
+constexpr int kQStages = 8;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
 constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
@@ -66,7 +66,8 @@ constexpr int kTileSlots = 4;
 constexpr int kConvWarps = 16;               // four per TMEM lane quarter
 constexpr int kConvGroups = kConvWarps / 4;  // warps of a quarter take turns: stage g goes to group g % 4
 constexpr int kEpiWarps = 8;
-constexpr int kThreads = (2 + kConvWarps + kEpiWarps) * 32;
+constexpr int kQWarp = 2 + kConvWarps + kEpiWarps;  // the weight-copy warp, after the epilogue warps
+constexpr int kThreads = (kQWarp + 1) * 32;
 constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
 constexpr int kQBytes = kWRows * kBK;       // 8 KB: int8 weights, 64-byte rows
 constexpr int kBarBytes = 512;
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < kTileSlots; ++s) {
             tc::mbar_init(&t_full[s], 1);
-            tc::mbar_init(&t_empty[s], 1 + kConvWarps + kEpiWarps);
+            tc::mbar_init(&t_empty[s], 2 + kConvWarps + kEpiWarps);  // MMA, converters, epilogue, weight copies
         }
         for (int b = 0; b < kAccBufs; ++b) {
             tc::mbar_init(&acc_full[b], 1);
@@ -242,12 +243,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     if (warp == 0) {
-        // ---------------- scheduler + TMA producer
+        // ---------------- scheduler + token-tile copies
         if (lane == 0) {
             int g = 0;
             Tile t;
+            // the next tile's index is claimed one tile ahead, so the atomic's latency hides
+            // behind the current tile's copies
+            int L_next = (int)blockIdx.x;
             for (int it = 0;; ++it) {
-                int L = (it == 0) ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(&p.hdr->sched[p.sched], 1);
+                int L = L_next;
                 if (L >= total || abort_flag) L = -1;
                 const int slot = it % kTileSlots, u = it / kTileSlots;
                 if (u > 0 && !tc::mbar_wait_bounded(&t_empty[slot], (u - 1) & 1, &abort_flag, p.max_polls)) {
@@ -257,12 +261,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tile_slot[slot] = L;
                 tc::mbar_arrive(&t_full[slot]);  // release: the slot write is visible to the waiters
                 if (L < 0) break;
+                L_next = (int)gridDim.x + atomicAdd(&p.hdr->sched[p.sched], 1);
                 tile_at(hdr, p, L, t);
-                const int w_row0 = t.e * p.N + t.n * (kDual ? kWRows / 2 : kWRows);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int sx = g % kXStages, rx = g / kXStages;
-                    const int sq = g % kQStages, rq = g / kQStages;
                     if (rx > 0 && !tc::mbar_wait_bounded(&x_empty[sx], (rx - 1) & 1, &abort_flag, p.max_polls)) {
                         ok = false;
                         break;
@@ -271,18 +274,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mbar_arrive_expect_tx(&x_full[sx], kXBytes);
                     tc::tma_load_2d(sX + sx * kXBytes, &tmX, &x_full[sx], kb * kBK, t.row0);
                     issued_x[sx] = rx;
+                }
+                if (!ok) {
+                    if (!abort_flag) fail(p.hdr, &abort_flag);
+                    break;
+                }
+            }
+        }
+    } else if (warp == kQWarp) {
+        // ---------------- int8 weight-tile copies, running ahead of the token copies as far as
+        // the (deeper) weight ring allows
+        if (lane == 0) {
+            int g = 0;
+            Tile t;
+            for (int it = 0;; ++it) {
+                const int L = next_tile(it);
+                if (L < 0) break;
+                tc::mbar_arrive(&t_empty[it % kTileSlots]);
+                tile_at(hdr, p, L, t);
+                const int w_row0 = t.e * p.N + t.n * (kDual ? kWRows / 2 : kWRows);
+                bool ok = true;
+                for (int kb = 0; kb < KB; ++kb, ++g) {
+                    const int sq = g % kQStages, rq = g / kQStages;
                     if (rq > 0 && !tc::mbar_wait_bounded(&q_empty[sq], (rq - 1) & 1, &abort_flag, p.max_polls)) {
                         ok = false;
                         break;
                     }
                     tc::mbar_arrive_expect_tx(&q_full[sq], kQBytes);
                     uint8_t* dq = sQ + sq * kQBytes;
-                    if (kDual) {
-                        tc::tma_load_2d(dq, &tmQ0, &q_full[sq], kb * kBK, w_row0);
-                        tc::tma_load_2d(dq + kQBytes / 2, &tmQ1, &q_full[sq], kb * kBK, w_row0);
-                    } else {
-                        tc::tma_load_2d(dq, &tmQ0, &q_full[sq], kb * kBK, w_row0);
-                    }
+                    tc::tma_load_2d(dq, &tmQ0, &q_full[sq], kb * kBK, w_row0);
+                    if (kDual) tc::tma_load_2d(dq + kQBytes / 2, &tmQ1, &q_full[sq], kb * kBK, w_row0);
                     issued_q[sq] = rq;
                 }
                 if (!ok) {
@@ -479,13 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::tc_fence_before();
     __syncthreads();
     if (abort_flag) {
+        // a copy of round r completes phase r of its full barrier; these waits ignore the abort flag
         if (warp == 0 && lane == 0) {
-            // a copy of round r completes phase r of its full barrier; these waits ignore the abort flag
             for (int s = 0; s < kXStages; ++s)
                 for (uint32_t i = 0; issued_x[s] >= 0 && i < p.max_polls &&
                                      !tc::mbar_try_wait(&x_full[s], issued_x[s] & 1);
                      ++i)
                     __nanosleep(64);
+        }
+        if (warp == kQWarp && lane == 0) {
             for (int s = 0; s < kQStages; ++s)
                 for (uint32_t i = 0; issued_q[s] >= 0 && i < p.max_polls &&
                                      !tc::mbar_try_wait(&q_full[s], issued_q[s] & 1);
