@@ -57,8 +57,8 @@ constexpr int kWRows = 128;   // weight rows per tile (MMA M, TMEM lanes)
 constexpr int kTokMax = 256;  // tokens per tile at most (MMA N)
 constexpr int kAccBufs = 1;   // TMEM accumulators (one of 256 columns leaves 256 for the weight ring)
 constexpr int kBK = 64;       // K elements per pipeline step
-constexpr int kXStages = 5;
-constexpr int kQStages = 8;
+constexpr int kXStages = 6;
+constexpr int kQStages = 4;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
 constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
@@ -69,6 +69,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kQWarp = 2 + kConvWarps + kEpiWarps;  // the weight-copy warp, after the epilogue warps
 constexpr int kThreads = (kQWarp + 1) * 32;
 constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
+constexpr int kXBoxRows = 32;                // rows of the copies that fill a partial token tile
 constexpr int kQBytes = kWRows * kBK;       // 8 KB: int8 weights, 64-byte rows
 constexpr int kBarBytes = 512;
 constexpr int kSmem = kXStages * kXBytes + kQStages * kQBytes + kBarBytes + 1024;
@@ -157,8 +158,8 @@ __device__ __forceinline__ int kpos(int k) { return (k & ~3) | ((k & 1) << 1) | 
 
 template <bool kDual>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_ts_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmQ0,
-                   const __grid_constant__ CUtensorMap tmQ1, Args p) {
+    gemm_ts_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmXs,
+                   const __grid_constant__ CUtensorMap tmQ0, const __grid_constant__ CUtensorMap tmQ1, Args p) {
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
@@ -215,6 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 0 && lane == 0) {
         tc::prefetch_tmap(&tmX);
+        tc::prefetch_tmap(&tmXs);
         tc::prefetch_tmap(&tmQ0);
         if (kDual) tc::prefetch_tmap(&tmQ1);
     }
@@ -263,6 +265,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (L < 0) break;
                 L_next = (int)gridDim.x + atomicAdd(&p.hdr->sched[p.sched], 1);
                 tile_at(hdr, p, L, t);
+                // a full tile takes one 256-row copy; a partial one only the 32-row boxes it uses
+                const int n_box = (t.ntok == kTokMax) ? 0 : (((t.ntok + 15) & ~15) + kXBoxRows - 1) / kXBoxRows;
+                const uint32_t x_bytes = n_box == 0 ? (uint32_t)kXBytes : (uint32_t)(n_box * kXBoxRows * 128);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int sx = g % kXStages, rx = g / kXStages;
@@ -271,8 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     if (p.skip_copy && blockIdx.x == 0 && it == 0 && kb == 1) continue;
-                    tc::mbar_arrive_expect_tx(&x_full[sx], kXBytes);
-                    tc::tma_load_2d(sX + sx * kXBytes, &tmX, &x_full[sx], kb * kBK, t.row0);
+                    tc::mbar_arrive_expect_tx(&x_full[sx], x_bytes);
+                    uint8_t* dx = sX + sx * kXBytes;
+                    if (n_box == 0) {
+                        tc::tma_load_2d(dx, &tmX, &x_full[sx], kb * kBK, t.row0);
+                    } else {
+                        for (int i = 0; i < n_box; ++i)
+                            tc::tma_load_2d(dx + i * kXBoxRows * 128, &tmXs, &x_full[sx], kb * kBK, t.row0 + i * kXBoxRows);
+                    }
                     issued_x[sx] = rx;
                 }
                 if (!ok) {
@@ -431,20 +442,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, L >= 0)) break;  // warp-uniform
             tile_at(hdr, p, L, t);
             const int b = it % kAccBufs, u = it / kAccBufs;
+            const int n_mma = (t.ntok + 15) & ~15;
+            constexpr int kChunks = kTokMax / 2 / 32;  // 32-token chunks of this warp's half of the tile
+            const int c0 = chalf * (kTokMax / 2);
+            // everything the epilogue needs besides the accumulator is loaded before waiting for it:
+            // the row scale and (W2) each chunk's assignment and routing weight for this lane's token
+            const int jl = 16 * qd + (lane & 15);  // W1/W3: lanes l and l + 16 hold gate and up of j0 + jl
+            const int il = 32 * qd + lane;         // W2: the output channel of this lane
+            const float sc = kDual ? __ldg((lane < 16 ? p.sa : p.sb) + (int64_t)t.e * p.N + t.n * (kWRows / 2) + jl)
+                                   : __ldg(p.sa + (int64_t)t.e * p.N + t.n * kWRows + il);
+            int32_t a_l[kChunks];
+            float w_l[kChunks];
+            if constexpr (!kDual) {
+#pragma unroll
+                for (int ci = 0; ci < kChunks; ++ci) {
+                    const int tok = c0 + 32 * ci + lane;
+                    a_l[ci] = (tok < t.ntok) ? p.perm[t.row0 + tok] : -1;
+                    w_l[ci] = a_l[ci] >= 0 ? p.wts[a_l[ci]] : 0.0f;
+                }
+            }
             bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, p.max_polls);
             if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
             if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
             tc::tc_fence_after();
             const uint32_t t_lane = t_quarter + (uint32_t)(b * kTokMax);
-            const int n_mma = (t.ntok + 15) & ~15;
             if constexpr (kDual) {
-                // lane l < 16: gate of j = j0 + 16 qd + l; lane l + 16: up of the same j
-                const int jl = 16 * qd + (lane & 15);
-                const int jg = t.n * (kWRows / 2) + jl;
-                const float sc = __ldg((lane < 16 ? p.sa : p.sb) + (int64_t)t.e * p.N + jg);
                 uint16_t* hcol = p.h_out + (int64_t)t.n * (kWRows / 2) + kpos(jl);
 #pragma unroll 1
-                for (int c = chalf * (kTokMax / 2); c < (chalf + 1) * (kTokMax / 2) && c < n_mma; c += 32) {
+                for (int c = c0; c < c0 + kTokMax / 2 && c < n_mma; c += 32) {
                     uint32_t v[32];
                     tc::tmem_ld32(t_lane + (uint32_t)c, v);
                     tc::tmem_wait_ld();
@@ -464,23 +489,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             } else {
-                const int il = 32 * qd + lane;
                 const int ig = t.n * kWRows + il;
-                const float s2 = __ldg(p.sa + (int64_t)t.e * p.N + ig);
-#pragma unroll 1
-                for (int c = chalf * (kTokMax / 2); c < (chalf + 1) * (kTokMax / 2) && c < n_mma; c += 32) {
+#pragma unroll
+                for (int ci = 0; ci < kChunks; ++ci) {
+                    const int c = c0 + 32 * ci;
+                    if (c >= n_mma) break;
                     uint32_t v[32];
                     tc::tmem_ld32(t_lane + (uint32_t)c, v);
-                    // this lane's token of the chunk: its assignment and routing weight
-                    const int32_t a_l = (c + lane < t.ntok) ? p.perm[t.row0 + c + lane] : -1;
-                    const float w_l = a_l >= 0 ? p.wts[a_l] : 0.0f;
                     tc::tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int32_t a = __shfl_sync(0xffffffffu, a_l, i);
-                        const float wt = __shfl_sync(0xffffffffu, w_l, i);
+                        const int32_t a = __shfl_sync(0xffffffffu, a_l[ci], i);
+                        const float wt = __shfl_sync(0xffffffffu, w_l[ci], i);
                         if (a >= 0) {
-                            const float o = wt * (s2 * __uint_as_float(v[i]));
+                            const float o = wt * (sc * __uint_as_float(v[i]));
                             if (p.y_out)
                                 p.y_out[(int64_t)(a / kTopK) * p.N + ig] = f32_to_bf16_bits(o);
                             else
@@ -577,8 +599,8 @@ int sm_count() {
 }
 
 template <bool kDual>
-cudaError_t launch(const CUtensorMap& tx, const CUtensorMap& tq0, const CUtensorMap& tq1, const Args& p,
-                   int64_t rows_cap, cudaStream_t st) {
+cudaError_t launch(const CUtensorMap& tx, const CUtensorMap& txs, const CUtensorMap& tq0, const CUtensorMap& tq1,
+                   const Args& p, int64_t rows_cap, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(gemm_ts_kernel<kDual>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (fewer when the row capacity allows fewer tiles)
@@ -586,7 +608,7 @@ cudaError_t launch(const CUtensorMap& tx, const CUtensorMap& tq0, const CUtensor
     const int sms = sm_count();
     if (grid > sms) grid = sms;
     if (grid < 1) grid = 1;
-    return launch_pdl(gemm_ts_kernel<kDual>, dim3((unsigned)grid), dim3(kThreads), kSmem, st, tx, tq0, tq1, p);
+    return launch_pdl(gemm_ts_kernel<kDual>, dim3((unsigned)grid), dim3(kThreads), kSmem, st, tx, txs, tq0, tq1, p);
 }
 
 int g_skip_copy = 0;  // set by jamba_moe_debug_skip_copy (tests only)
@@ -599,8 +621,10 @@ cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_
                           const float* S1, const int8_t* Q3, const float* S3, uint16_t* h, int64_t rows_cap,
                           int64_t d, int64_t F, cudaStream_t st, int n_exp) {
     using namespace ts;
-    CUtensorMap tx, tq0, tq1;
+    CUtensorMap tx, txs, tq0, tq1;
     if (!make_map(&tx, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kTokMax, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&txs, x_perm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, d, kXBoxRows, kBK,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tq0, Q1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * F, d, kWRows / 2, kBK,
                   CU_TENSOR_MAP_SWIZZLE_64B) ||
@@ -620,7 +644,7 @@ cudaError_t launch_gemm13(WsHeader* hdr, const int32_t* perm, const uint16_t* x_
     p.sched = 0;
     p.max_polls = g_skip_copy ? kTestMaxPolls : kMaxPolls;
     p.skip_copy = g_skip_copy;
-    return launch<true>(tx, tq0, tq1, p, rows_cap, st);
+    return launch<true>(tx, txs, tq0, tq1, p, rows_cap, st);
 }
 
 // out_slot[a] = p_a * S2 . (h_perm . Q2^T) per expert segment, or, given y (the dense MLP, one
@@ -629,8 +653,10 @@ cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, 
                          const float* wts, float* out_slot, int64_t rows_cap, int64_t d, int64_t F, cudaStream_t st,
                          int n_exp, uint16_t* y) {
     using namespace ts;
-    CUtensorMap tx, tq0;
+    CUtensorMap tx, txs, tq0;
     if (!make_map(&tx, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kTokMax, kBK,
+                  CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&txs, h, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows_cap, F, kXBoxRows, kBK,
                   CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&tq0, Q2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)n_exp * d, F, kWRows, kBK,
                   CU_TENSOR_MAP_SWIZZLE_64B))
@@ -649,7 +675,7 @@ cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, 
     p.sched = 1;
     p.max_polls = g_skip_copy ? kTestMaxPolls : kMaxPolls;
     p.skip_copy = 0;
-    return launch<false>(tx, tq0, tq0, p, rows_cap, st);
+    return launch<false>(tx, txs, tq0, tq0, p, rows_cap, st);
 }
 
 }  // namespace jmoe
