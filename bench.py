@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.ALL_WORKLOADS),
                     help="MoE layer workloads, or mlp_* for the dense ExpertsInt8 MLP")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="run the workload's layer shape on this many tokens instead of its own T")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--path", default="auto", choices=["auto", "gemv", "gemm"])
     ap.add_argument("--weights", default="int8", choices=["int8", "bf16", "fp8"],
@@ -266,7 +268,7 @@ def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
         return 0
-    wl = synth.ALL_WORKLOADS[args.workload]
+    wl = workload_of(args)
     setup = oracle_setup(wl, wl.seed)
     import oracle
     threads = oracle.default_threads()
@@ -296,6 +298,12 @@ def run_reference(args):
     }
     print(json.dumps(out), flush=True)
     return 0
+
+
+def workload_of(args):
+    """The named workload, with its token count replaced when --tokens is given."""
+    wl = synth.ALL_WORKLOADS[args.workload]
+    return synth_replace(wl, T=args.tokens) if args.tokens else wl
 
 
 def run_config(wl, args, world):
@@ -364,7 +372,7 @@ def run_ours(args):
             os.environ.setdefault("RANK", "0")
             os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    wl = synth.ALL_WORKLOADS[args.workload]
+    wl = workload_of(args)
     mlp = wl.layer == "mlp"
     if mlp and args.weights != "int8":
         raise SystemExit("the dense MLP workloads run with ExpertsInt8 weights only")
