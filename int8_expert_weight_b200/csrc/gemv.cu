@@ -201,7 +201,7 @@ __device__ __forceinline__ void gemv_pass(const GemvArgs& p, int e, int64_t j0, 
 
 template <int NT, bool kDual, bool kW8>
 __global__ void __launch_bounds__(kGemvWarps * 32,
-                                  kW8 ? ((NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? ((kDual) ? 2 : 4) : 1))
+                                  kW8 ? ((NT == 1) ? ((kDual) ? 3 : 4) : (NT <= 2 ? ((kDual) ? 2 : 4) : 2))
                                       : ((NT == 1) ? 2 : 1))
     gemv_kernel(GemvArgs p) {
     __shared__ __align__(16) float red[kGemvWarps * 2 * NT * 128];
@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32,
         }
         // W2 with 16 tokens per pass: one k-step in flight per warp and 4 CTAs per SM stream faster
         // than two steps at 2 CTAs per SM
-        gemv_pass<NT, kDual, kW8, (kW8 && !kDual && NT == 2) ? 1 : 2>(p, e, j0, rows, red);
+        gemv_pass<NT, kDual, kW8, (kW8 && ((!kDual && NT == 2) || NT == 4)) ? 1 : 2>(p, e, j0, rows, red);
         pdl_trigger();  // main loop done: the next kernel may start launching
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
