@@ -592,6 +592,10 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
     if world > 1:
         dist.destroy_process_group()
+    bad = {k: v for k, v in status.items() if v != 0}
+    if bad:  # a bounded wait ran out or a kernel skipped a bad index: the numbers above are void
+        print(f"rank {rank}: device status {bad} ({jm.jamba_moe_status_string(max(bad.values()))})", file=sys.stderr)
+        return 3
     return 0
 
 
