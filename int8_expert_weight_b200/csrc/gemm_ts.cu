@@ -18,18 +18,22 @@
 // the converters read the int8 tile from shared memory and write BF16 pairs straight into TMEM
 // with tcgen05.st, from where the MMA reads them.
 //
-// Persistent, one CTA per SM, 576 threads in roles:
-//   warp 0       producer: tile scheduler (first tile = CTA index, then an atomic counter in the
-//                workspace header) and TMA copies: token tile bf16 [256][64] SWIZZLE_128B,
-//                int8 weight tile [128][64] SWIZZLE_64B, per 64-wide K step
+// Persistent, one CTA per SM, 864 threads in roles:
+//   warp 0       tile scheduler (first tile = CTA index, then an atomic counter in the workspace
+//                header, claimed one tile ahead) and token copies: TMA of the bf16 token tile
+//                [256][64] SWIZZLE_128B per 64-wide K step (a partial tile: only its 32-row boxes)
+//   warp 26      int8 weight copies: TMA of the tile [128][64] SWIZZLE_64B per K step
 //   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16, A from TMEM, B from smem,
 //                M = 128, N = tokens of the tile rounded up to 16, K = 16
-//   warps 2-9    converters: int8 -> bf16 (exact), two warps per TMEM lane quarter, each 32 of the
-//                64 K of a step; tcgen05.st into an 8-stage TMEM ring
-//   warps 10-17  epilogue: tcgen05.ld of the accumulator, two warps per lane quarter (128 tokens
-//                each), scales, SiLU * up or routing weight, global stores
+//   warps 2-9    converters: int8 -> bf16 (exact), two warps per TMEM lane quarter taking turns
+//                by K step; each converts the 64 K of its 32 rows and stores them with tcgen05.st
+//                into an 8-stage TMEM ring
+//   warps 10-25  epilogue: tcgen05.ld of the accumulator, four warps per lane quarter (64 tokens
+//                each), scales, SiLU * up or routing weight, global stores.  The MMA of the next
+//                tile waits until the accumulator is read out, so the epilogue is split over
+//                as many warps as the register budget allows
 // TMEM: 256 accumulator columns (fp32 [128][256]) + 256 columns of converted weights (8 stages of
-// 32 columns = 64 bf16 per lane).  Rings: 5 token stages, 6 int8 stages, 8 TMEM stages, 4 tile
+// 32 columns = 64 bf16 per lane).  Rings: 6 token stages, 4 int8 stages, 8 TMEM stages, 4 tile
 // slots.  Every mbarrier wait is bounded: on timeout the kernel records JMOE_DEV_TIMEOUT in the
 // workspace status word, the other roles stop at their next wait, in-flight copies and MMAs are
 // waited for (bounded), TMEM is released and the CTA returns.
@@ -63,9 +67,11 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
 constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
 constexpr int kTileSlots = 4;
-constexpr int kConvWarps = 16;               // four per TMEM lane quarter
-constexpr int kConvGroups = kConvWarps / 4;  // warps of a quarter take turns: stage g goes to group g % 4
-constexpr int kEpiWarps = 8;
+constexpr int kConvWarps = 8;                // two per TMEM lane quarter
+constexpr int kConvGroups = kConvWarps / 4;  // warps of a quarter take turns: stage g goes to group g % 2
+constexpr int kEpiWarps = 16;                // four per TMEM lane quarter
+constexpr int kEpiParts = kEpiWarps / 4;     // column ranges of the accumulator, one per warp of a quarter
+constexpr int kEpiCols = kTokMax / kEpiParts;
 constexpr int kQWarp = 2 + kConvWarps + kEpiWarps;  // the weight-copy warp, after the epilogue warps
 constexpr int kThreads = (kQWarp + 1) * 32;
 constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ---------------- epilogue
-        const int ew = warp - 2 - kConvWarps, qd = warp & 3, chalf = ew >> 2;
+        const int ew = warp - 2 - kConvWarps, qd = warp & 3, cpart = ew >> 2;
         const uint32_t t_quarter = tmem + ((uint32_t)(32 * qd) << 16);
         Tile t;
         for (int it = 0;; ++it) {
@@ -443,8 +449,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             tile_at(hdr, p, L, t);
             const int b = it % kAccBufs, u = it / kAccBufs;
             const int n_mma = (t.ntok + 15) & ~15;
-            constexpr int kChunks = kTokMax / 2 / 32;  // 32-token chunks of this warp's half of the tile
-            const int c0 = chalf * (kTokMax / 2);
+            constexpr int kChunks = kEpiCols / 32;  // 32-token chunks of this warp's part of the tile
+            const int c0 = cpart * kEpiCols;
             // everything the epilogue needs besides the accumulator is loaded before waiting for it:
             // the row scale and (W2) each chunk's assignment and routing weight for this lane's token
             const int jl = 16 * qd + (lane & 15);  // W1/W3: lanes l and l + 16 hold gate and up of j0 + jl
@@ -469,7 +475,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (kDual) {
                 uint16_t* hcol = p.h_out + (int64_t)t.n * (kWRows / 2) + kpos(jl);
 #pragma unroll 1
-                for (int c = c0; c < c0 + kTokMax / 2 && c < n_mma; c += 32) {
+                for (int c = c0; c < c0 + kEpiCols && c < n_mma; c += 32) {
                     uint32_t v[32];
                     tc::tmem_ld32(t_lane + (uint32_t)c, v);
                     tc::tmem_wait_ld();
