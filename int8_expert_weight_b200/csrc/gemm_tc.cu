@@ -7,8 +7,10 @@
 //           the same 128 j of W3), so both halves of SwiGLU meet in one accumulator
 //   gemm2:  out[a][i] = p_a * (h_r . W2[i])                         tile: 128 rows x BN i
 //
-// Persistent: one CTA per SM walks the tile list with stride gridDim.x; 192 threads in roles:
-//   warp 0       TMA producer: activation tile + weight tile per K step, both straight into the
+// Persistent: one CTA per SM; 192 threads in roles:
+//   warp 0       tile scheduler (first tile = CTA index, then an atomic counter in the workspace
+//                header, claimed one tile ahead and published through a 4-slot ring) and TMA
+//                producer: activation tile + weight tile per K step, both straight into the
 //                MMA's SWIZZLE_128B K-major layout (128 bytes of K per row)
 //   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16 (bf16) or kind::f8f6f4 (E4M3),
 //                M=128, N=BN, fp32 accumulators in TMEM
@@ -20,7 +22,9 @@
 // for (bounded), TMEM is released and the CTA returns.
 //
 // Tiles are ordered expert by expert; inside an expert, bands of M tiles keep their activations
-// resident in L2 while every N tile of the weights streams past once per band.
+// resident in L2 while every N tile of the weights streams past once per band.  Tiles are handed
+// out in list order as CTAs become free (not by a fixed stride), so the CTAs that share a weight
+// tile start it together and read it while it is still in L2.
 //
 // FP8 (kF8): E4M3 activations and weights, 128 K elements per stage, kind::f8f6f4 MMAs, per-row
 // activation scales and per-channel weight scales in the epilogue, bf16 h.
@@ -55,7 +59,9 @@ struct GemmArgs {
     // FP8 layer only: per-row activation scale (gemm13: per token, indexed by assignment / K;
     // gemm2: per permuted row)
     const float* a_scale;
+    int sched;  // which tile counter of the header this GEMM uses (zeroed by the permutation)
 };
+constexpr int kTileSlots = 4;
 
 // Shared-memory ring: per stage the activation tile and the weight tile, both as the MMA reads
 // them (128 bytes of K per row: 64 bf16 or 128 E4M3).
@@ -112,6 +118,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint32_t tmem_holder;
     __shared__ volatile int abort_flag;
+    __shared__ volatile int tile_slot[kTileSlots];
 
     pdl_wait();
     const WsHeader* hdr = p.hdr;
@@ -125,6 +132,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t* acc_full = bars + 2 * kStages;    // [2] accumulator complete
     uint64_t* acc_empty = acc_full + 2;         // [2] accumulator read out by the epilogue
     uint64_t* mma_done = acc_empty + 2;         // every issued MMA complete (teardown)
+    uint64_t* t_full = mma_done + 1;            // [kTileSlots] tile index published
+    uint64_t* t_empty = t_full + kTileSlots;    // [kTileSlots] read by the MMA and epilogue warps
+    static_assert((2 * kStages + 5 + 2 * kTileSlots) * 8 <= 256, "barriers");
     auto sA = [&](int s) { return smem + s * SL::kStage; };
     auto sB = [&](int s) { return smem + s * SL::kStage + SL::kA; };
 
@@ -139,6 +149,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tc::mbar_init(&acc_empty[b], kEpiWarps);
         }
         tc::mbar_init(mma_done, 1);
+        for (int s = 0; s < kTileSlots; ++s) {
+            tc::mbar_init(&t_full[s], 1);
+            tc::mbar_init(&t_empty[s], 1 + kEpiWarps);
+        }
         abort_flag = 0;
         tc::mbar_fence_init();
     }
@@ -162,12 +176,36 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int s = 0; s < kStages; ++s) issued_round[s] = -1;
     int mma_issued = 0;
 
+    // MMA and epilogue warps: the index of tile `it` (-1 past the last), or -2 after an abort.
+    auto next_tile = [&](int it) -> int {
+        const int slot = it % kTileSlots, u = it / kTileSlots;
+        if (!tc::mbar_wait_bounded(&t_full[slot], u & 1, &abort_flag, p.max_polls)) {
+            if (!abort_flag) fail(p.hdr, &abort_flag);
+            return -2;
+        }
+        return tile_slot[slot];
+    };
+
     if (warp == 0) {
-        // ---------------- TMA producer
+        // ---------------- tile scheduler + TMA producer
         if (lane == 0) {
             int g = 0;
             TileCoord t;
-            for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x) {
+            // the next tile's index is claimed one tile ahead, so the atomic's latency hides behind
+            // the current tile's copies
+            int L_next = (int)blockIdx.x;
+            for (int it = 0;; ++it) {
+                int L = L_next;
+                if (L >= total || abort_flag) L = -1;
+                const int slot = it % kTileSlots, u = it / kTileSlots;
+                if (u > 0 && !tc::mbar_wait_bounded(&t_empty[slot], (u - 1) & 1, &abort_flag, p.max_polls)) {
+                    if (!abort_flag) fail(p.hdr, &abort_flag);
+                    break;
+                }
+                tile_slot[slot] = L;
+                tc::mbar_arrive(&t_full[slot]);  // release: the slot write is visible to the waiters
+                if (L < 0) break;
+                L_next = (int)gridDim.x + atomicAdd(&p.hdr->sched[p.sched], 1);
                 tile_coord(hdr, p, L, t);
                 const int a_row0 = hdr->seg_start[t.e] + t.m_tile * kBM;
                 const int w_row0 = t.e * p.N + t.n_tile * (kDual ? BN / 2 : BN);
@@ -191,8 +229,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         // ---------------- MMA issuer
         if (lane == 0) {
-            int g = 0, it = 0;
-            for (int L = blockIdx.x; L < total && !abort_flag; L += gridDim.x, ++it) {
+            int g = 0;
+            for (int it = 0;; ++it) {
+                const int L = next_tile(it);
+                if (L < 0) break;
+                tc::mbar_arrive(&t_empty[it % kTileSlots]);
                 const int b = it & 1, u = it >> 1;
                 if (u > 0 && !tc::mbar_wait_bounded(&acc_empty[b], (u - 1) & 1, &abort_flag, p.max_polls)) {
                     if (!abort_flag) fail(p.hdr, &abort_flag);
@@ -231,10 +272,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // ---------------- epilogue
         const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
         const int row = q * 32 + lane;
-        int it = 0;
         TileCoord t;
-        for (int L = blockIdx.x; L < total; L += gridDim.x, ++it) {
-            if (__any_sync(0xffffffffu, abort_flag != 0)) break;  // warp-uniform
+        for (int it = 0;; ++it) {
+            const int L = next_tile(it);
+            __syncwarp();
+            if (lane == 0 && L >= 0) tc::mbar_arrive(&t_empty[it % kTileSlots]);
+            if (!__all_sync(0xffffffffu, L >= 0)) break;  // warp-uniform
             const int b = it & 1, u = it >> 1;
             bool ok = tc::mbar_wait_bounded(&acc_full[b], u & 1, &abort_flag, p.max_polls);
             if (!ok && !abort_flag) fail(p.hdr, &abort_flag);
@@ -276,8 +319,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
             } else if (kDual) {
                 const int j0 = t.n_tile * (BN / 2);
-                const float* s1 = p.sa + (int64_t)t.e * p.N + j0;
-                const float* s3 = p.sb + (int64_t)t.e * p.N + j0;
                 uint16_t* hrow = p.h_out + gr * p.N + j0;
 #pragma unroll 1
                 for (int c = 0; c < BN / 2; c += 32) {
@@ -436,7 +477,7 @@ cudaError_t launch_gemm13_bf16w(WsHeader* hdr, const int32_t* perm, const uint16
     GemmArgs p{hdr,          perm,          nullptr,     nullptr,
                nullptr,      h,             nullptr,     (int)d,
                (int)F,       (int)(F / 128), band_for((int)d, 2), kMaxPolls,
-               nullptr};
+               nullptr,      0};
     return launch_gemm_t<true, 256, false>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
@@ -452,7 +493,7 @@ cudaError_t launch_gemm2_bf16w(WsHeader* hdr, const int32_t* perm, const uint16_
     GemmArgs p{hdr,         perm,         nullptr,     nullptr,
                wts,         nullptr,      out_slot,    (int)F,
                (int)d,      (int)(d / BN), band_for((int)F, 2), kMaxPolls,
-               nullptr};
+               nullptr,     1};
     if (BN == 256) return launch_gemm_t<false, 256, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128, false>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
@@ -472,7 +513,7 @@ cudaError_t launch_gemm13_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* 
     GemmArgs p{hdr,          perm,          S1,          S3,
                nullptr,      h,             nullptr,     (int)d,
                (int)F,       (int)(F / 128), band_for((int)d, 1), kMaxPolls,
-               sx};
+               sx,           0};
     return launch_gemm_t<true, 256, true>(ta, tb0, tb1, p, rows_cap / kBM, st);
 }
 
@@ -489,7 +530,7 @@ cudaError_t launch_gemm2_f8(WsHeader* hdr, const int32_t* perm, const uint8_t* h
     GemmArgs p{hdr,         perm,         S2,          nullptr,
                wts,         nullptr,      out_slot,    (int)F,
                (int)d,      (int)(d / BN), band_for((int)F, 1), kMaxPolls,
-               sh};
+               sh,          1};
     if (BN == 256) return launch_gemm_t<false, 256, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
     return launch_gemm_t<false, 128, true>(ta, tb0, tb0, p, rows_cap / kBM, st);
 }
