@@ -472,13 +472,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__all_sync(0xffffffffu, ok)) break;  // tcgen05.ld below is warp-collective
             tc::tc_fence_after();
             const uint32_t t_lane = t_quarter + (uint32_t)(b * kTokMax);
+            // the accumulator is released as soon as this warp's last chunk is in registers, so the
+            // next tile's MMAs overlap the math and stores of that chunk
+            const int c_end = min(c0 + kEpiCols, n_mma);
+            bool released = false;
+            auto release = [&]() {
+                tc::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
+                released = true;
+            };
             if constexpr (kDual) {
                 uint16_t* hcol = p.h_out + (int64_t)t.n * (kWRows / 2) + kpos(jl);
 #pragma unroll 1
-                for (int c = c0; c < c0 + kEpiCols && c < n_mma; c += 32) {
+                for (int c = c0; c < c_end; c += 32) {
                     uint32_t v[32];
                     tc::tmem_ld32(t_lane + (uint32_t)c, v);
                     tc::tmem_wait_ld();
+                    if (c + 32 >= c_end) release();
                     // lanes < 16 keep the gate of tokens c .. c+15 and take the up values from lane + 16;
                     // lanes >= 16 keep the up of tokens c+16 .. c+31 and take the gate values from lane - 16
                     const int tok0 = c + ((lane < 16) ? 0 : 16);
@@ -503,6 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t v[32];
                     tc::tmem_ld32(t_lane + (uint32_t)c, v);
                     tc::tmem_wait_ld();
+                    if (c + 32 >= c_end) release();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         const int32_t a = __shfl_sync(0xffffffffu, a_l[ci], i);
@@ -517,9 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            tc::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&acc_empty[b]);
+            if (!released) release();  // a warp whose columns hold no tokens of this tile
         }
     }
 
