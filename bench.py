@@ -428,7 +428,7 @@ def run_ours(args):
     ep_steps = CudaSteps(path) if ep else None
     y_ep = [y]
 
-    def forward(xin):
+    def forward(xin, y=y):
         if ep:
             y_ep[0], ids_ep, _ = ep_forward(xin, wr, bias, (Q["w1"], S["w1"], Q["w3"], S["w3"], Q["w2"], S["w2"]),
                                             steps=ep_steps, stats=ep_stats)
@@ -505,24 +505,54 @@ def run_ours(args):
     ms_events = max_over_ranks(ms_events, dev)
     value = aggregate_tokens_per_s(world, T, args.steps, ms)
 
-    # ---- end to end through the public call with host buffers: pinned x in, pinned y out
+    # ---- end to end through the public call with host buffers: pinned x in, pinned y out.  Every
+    # step copies its x from pinned host memory and its y back; the copies run on their own
+    # streams (one per direction) with two device buffers, so step i+1's input copy and step i-1's
+    # output copy overlap step i's layer, as a serving loop would.  The expert-parallel path keeps
+    # the plain sequential loop (its outputs are allocated by the exchange).
     x_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
     x_host.copy_(x.cpu())
     y_host = torch.empty((T, d), dtype=torch.bfloat16, pin_memory=True)
-    x_dev = torch.empty_like(x)
+    x_dev = [torch.empty_like(x) for _ in range(2)]
+    y_dev = [y, torch.empty_like(y)]
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def step_e2e():
-        x_dev.copy_(x_host, non_blocking=True)
-        forward(x_dev)
-        y_host.copy_(y_ep[0] if ep else y, non_blocking=True)
+    def e2e_steps(n):
+        """n steps; ends with the compute stream waiting for the last output copy."""
+        for i in range(n):
+            b = i & 1
+            if ep:
+                x_dev[0].copy_(x_host, non_blocking=True)
+                forward(x_dev[0])
+                y_host.copy_(y_ep[0], non_blocking=True)
+                continue
+            if i == 0:
+                s_in.wait_stream(stream)  # the first copy starts after the timing event
+            elif i >= 2:
+                s_in.wait_event(ev_done[b])  # step i-2's layer has read x_dev[b]
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+                ev_in[b].record(s_in)
+            stream.wait_event(ev_in[b])
+            if i >= 2:
+                stream.wait_event(ev_out[b])  # step i-2's output copy has left y_dev[b]
+            forward(x_dev[b], y_dev[b])
+            ev_done[b].record(stream)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                y_host.copy_(y_dev[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        if not ep and n > 0:
+            stream.wait_event(ev_out[(n - 1) & 1])
 
-    for _ in range(args.warmup):
-        step_e2e()
+    e2e_steps(args.warmup)
     torch.cuda.synchronize()
     barrier()
     ev0.record(stream)
-    for _ in range(args.steps):
-        step_e2e()
+    e2e_steps(args.steps)
     ev1.record(stream)
     torch.cuda.synchronize()
     status["e2e"] = read_status()
