@@ -18,25 +18,27 @@
 // the converters read the int8 tile from shared memory and write BF16 pairs straight into TMEM
 // with tcgen05.st, from where the MMA reads them.
 //
-// Persistent, one CTA per SM, 864 threads in roles:
+// Persistent, one CTA per SM, 864 threads in roles.  A pipeline stage covers 128 of K as two
+// 64-wide sub-steps: every hand-off between the roles (copy landed, weights converted, MMAs done)
+// is one mbarrier round trip per 128 K, whose fixed latency would otherwise set the pace.
 //   warp 0       tile scheduler (first tile = CTA index, then an atomic counter in the workspace
-//                header, claimed one tile ahead) and token copies: TMA of the bf16 token tile
-//                [256][64] SWIZZLE_128B per 64-wide K step (a partial tile: only its 32-row boxes)
-//   warp 26      int8 weight copies: TMA of the tile [128][64] SWIZZLE_64B per K step
+//                header, claimed one tile ahead) and token copies: per stage two TMA boxes of the
+//                bf16 token tile [256][64] SWIZZLE_128B (a partial tile: only its 32-row boxes)
+//   warp 26      int8 weight copies: per stage two TMA boxes of the tile [128][64] SWIZZLE_64B
 //   warp 1       TMEM allocator and MMA issuer: tcgen05.mma kind::f16, A from TMEM, B from smem,
-//                M = 128, N = tokens of the tile rounded up to 16, K = 16
+//                M = 128, N = tokens of the tile rounded up to 16, K = 16 (8 per stage)
 //   warps 2-9    converters: int8 -> bf16 (exact), two warps per TMEM lane quarter taking turns
-//                by K step; each converts the 64 K of its 32 rows and stores them with tcgen05.st
-//                into an 8-stage TMEM ring
+//                by stage; each converts the 128 K of its 32 rows and stores them with tcgen05.st
+//                into a 4-stage TMEM ring
 //   warps 10-25  epilogue: tcgen05.ld of the accumulator, four warps per lane quarter (64 tokens
 //                each), scales, SiLU * up or routing weight, global stores.  The MMA of the next
 //                tile waits until the accumulator is read out, so the epilogue is split over
 //                as many warps as the register budget allows
-// TMEM: 256 accumulator columns (fp32 [128][256]) + 256 columns of converted weights (8 stages of
-// 32 columns = 64 bf16 per lane).  Rings: 6 token stages, 4 int8 stages, 8 TMEM stages, 4 tile
-// slots.  Every mbarrier wait is bounded: on timeout the kernel records JMOE_DEV_TIMEOUT in the
-// workspace status word, the other roles stop at their next wait, in-flight copies and MMAs are
-// waited for (bounded), TMEM is released and the CTA returns.
+// TMEM: 256 accumulator columns (fp32 [128][256]) + 256 columns of converted weights (4 stages of
+// 64 columns = 128 bf16 per lane).  Rings: 3 token stages (64 KB each), 2 int8 stages (16 KB),
+// 4 TMEM stages, 4 tile slots.  Every mbarrier wait is bounded: on timeout the kernel records
+// JMOE_DEV_TIMEOUT in the workspace status word, the other roles stop at their next wait,
+// in-flight copies and MMAs are waited for (bounded), TMEM is released and the CTA returns.
 //
 // Tile order: expert by expert; inside an expert, bands of token tiles whose activations stay in
 // L2 while every weight tile streams past once per band; token tiles fastest inside a band, so the
@@ -60,12 +62,13 @@ namespace ts {
 constexpr int kWRows = 128;   // weight rows per tile (MMA M, TMEM lanes)
 constexpr int kTokMax = 256;  // tokens per tile at most (MMA N)
 constexpr int kAccBufs = 1;   // TMEM accumulators (one of 256 columns leaves 256 for the weight ring)
-constexpr int kBK = 64;       // K elements per pipeline step
-constexpr int kXStages = 6;
-constexpr int kQStages = 4;
+constexpr int kBK = 64;       // K elements per copy box and converted sub-step
+constexpr int kSub = 2;       // sub-steps per pipeline stage (one barrier hand-off per 128 K)
+constexpr int kXStages = 3;
+constexpr int kQStages = 2;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kACol0 = kAccBufs * kTokMax;  // first TMEM column of the converted-weight ring
-constexpr int kAStages = (int)(kTmemCols - kACol0) / 32;  // 32 columns = 64 bf16 per lane per stage
+constexpr int kAStages = (int)(kTmemCols - kACol0) / (32 * kSub);  // 32 columns = 64 bf16 per lane per sub-step
 constexpr int kTileSlots = 4;
 constexpr int kConvWarps = 8;                // two per TMEM lane quarter
 constexpr int kConvGroups = kConvWarps / 4;  // warps of a quarter take turns: stage g goes to group g % 2
@@ -74,9 +77,11 @@ constexpr int kEpiParts = kEpiWarps / 4;     // column ranges of the accumulator
 constexpr int kEpiCols = kTokMax / kEpiParts;
 constexpr int kQWarp = 2 + kConvWarps + kEpiWarps;  // the weight-copy warp, after the epilogue warps
 constexpr int kThreads = (kQWarp + 1) * 32;
-constexpr int kXBytes = kTokMax * kBK * 2;  // bf16 tokens, 128-byte rows
+constexpr int kXSub = kTokMax * kBK * 2;  // bf16 tokens of one sub-step, 128-byte rows
+constexpr int kXBytes = kSub * kXSub;
 constexpr int kXBoxRows = 32;                // rows of the copies that fill a partial token tile
-constexpr int kQBytes = kWRows * kBK;       // 8 KB: int8 weights, 64-byte rows
+constexpr int kQSub = kWRows * kBK;       // 8 KB: int8 weights of one sub-step, 64-byte rows
+constexpr int kQBytes = kSub * kQSub;
 constexpr int kBarBytes = 512;
 constexpr int kSmem = kXStages * kXBytes + kQStages * kQBytes + kBarBytes + 1024;
 constexpr uint32_t kMaxPolls = 1u << 22;      // ~0.3 s of polling: far above any healthy wait
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::tc_fence_after();
     const uint32_t tmem = tmem_holder;
-    const int KB = p.K / kBK;
+    const int KB = p.K / (kBK * kSub);
     int issued_x[kXStages], issued_q[kQStages];  // producer: last round issued on each stage (-1: none)
 #pragma unroll
     for (int s = 0; s < kXStages; ++s) issued_x[s] = -1;
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tile_at(hdr, p, L, t);
                 // a full tile takes one 256-row copy; a partial one only the 32-row boxes it uses
                 const int n_box = (t.ntok == kTokMax) ? 0 : (((t.ntok + 15) & ~15) + kXBoxRows - 1) / kXBoxRows;
-                const uint32_t x_bytes = n_box == 0 ? (uint32_t)kXBytes : (uint32_t)(n_box * kXBoxRows * 128);
+                const uint32_t x_bytes = n_box == 0 ? (uint32_t)kXBytes : (uint32_t)(kSub * n_box * kXBoxRows * 128);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb, ++g) {
                     const int sx = g % kXStages, rx = g / kXStages;
@@ -283,12 +288,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (p.skip_copy && blockIdx.x == 0 && it == 0 && kb == 1) continue;
                     tc::mbar_arrive_expect_tx(&x_full[sx], x_bytes);
-                    uint8_t* dx = sX + sx * kXBytes;
-                    if (n_box == 0) {
-                        tc::tma_load_2d(dx, &tmX, &x_full[sx], kb * kBK, t.row0);
-                    } else {
-                        for (int i = 0; i < n_box; ++i)
-                            tc::tma_load_2d(dx + i * kXBoxRows * 128, &tmXs, &x_full[sx], kb * kBK, t.row0 + i * kXBoxRows);
+                    for (int sub = 0; sub < kSub; ++sub) {
+                        uint8_t* dx = sX + sx * kXBytes + sub * kXSub;
+                        const int kx = (kb * kSub + sub) * kBK;
+                        if (n_box == 0) {
+                            tc::tma_load_2d(dx, &tmX, &x_full[sx], kx, t.row0);
+                        } else {
+                            for (int i = 0; i < n_box; ++i)
+                                tc::tma_load_2d(dx + i * kXBoxRows * 128, &tmXs, &x_full[sx], kx, t.row0 + i * kXBoxRows);
+                        }
                     }
                     issued_x[sx] = rx;
                 }
@@ -318,9 +326,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc::mbar_arrive_expect_tx(&q_full[sq], kQBytes);
-                    uint8_t* dq = sQ + sq * kQBytes;
-                    tc::tma_load_2d(dq, &tmQ0, &q_full[sq], kb * kBK, w_row0);
-                    if (kDual) tc::tma_load_2d(dq + kQBytes / 2, &tmQ1, &q_full[sq], kb * kBK, w_row0);
+                    for (int sub = 0; sub < kSub; ++sub) {
+                        uint8_t* dq = sQ + sq * kQBytes + sub * kQSub;
+                        const int kx = (kb * kSub + sub) * kBK;
+                        tc::tma_load_2d(dq, &tmQ0, &q_full[sq], kx, w_row0);
+                        if (kDual) tc::tma_load_2d(dq + kQSub / 2, &tmQ1, &q_full[sq], kx, w_row0);
+                    }
                     issued_q[sq] = rq;
                 }
                 if (!ok) {
@@ -359,11 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     tc::tc_fence_after();
-                    const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sX + sx * kXBytes));
-                    const uint32_t a_col = tmem + kACol0 + (uint32_t)(sa * 32);
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)  // 16 bf16 = 8 TMEM columns of A, 32 bytes of B
-                        tc::mma_bf16_ts(d_tmem, a_col + 8 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
+                    for (int sub = 0; sub < kSub; ++sub) {
+                        const uint64_t bdesc = tc::sw128_kmajor_desc(tc::smem_u32(sX + sx * kXBytes + sub * kXSub));
+                        const uint32_t a_col = tmem + kACol0 + (uint32_t)(sa * 32 * kSub + sub * 32);
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk)  // 16 bf16 = 8 TMEM columns of A, 32 bytes of B
+                            tc::mma_bf16_ts(d_tmem, a_col + 8 * kk, bdesc + 2 * kk, idesc, (kb | sub | kk) != 0);
+                    }
                     tc::mma_commit(&x_empty[sx]);
                     tc::mma_commit(&a_empty[sa]);
                     ++mma_issued;
@@ -404,31 +418,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 const uint8_t* q8 = sQ + sq * kQBytes;
-                uint4 v[4];
+                bool free_ = true;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(q8 + coff[i]);
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&q_empty[sq]);
-                uint32_t o0[16], o1[16];
+                for (int sub = 0; sub < kSub; ++sub) {
+                    uint4 v[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t* o = (i < 2) ? o0 : o1;
-                        o[8 * (i & 1) + 2 * j] = s8x2_even_to_bf16x2(w[j], k8);
-                        o[8 * (i & 1) + 2 * j + 1] = s8x2_odd_to_bf16x2(w[j], k8);
+                    for (int i = 0; i < 4; ++i) v[i] = *reinterpret_cast<const uint4*>(q8 + sub * kQSub + coff[i]);
+                    if (sub == kSub - 1) {
+                        __syncwarp();
+                        if (lane == 0) tc::mbar_arrive(&q_empty[sq]);
                     }
+                    uint32_t o0[16], o1[16];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint32_t* o = (i < 2) ? o0 : o1;
+                            o[8 * (i & 1) + 2 * j] = s8x2_even_to_bf16x2(w[j], k8);
+                            o[8 * (i & 1) + 2 * j + 1] = s8x2_odd_to_bf16x2(w[j], k8);
+                        }
+                    }
+                    if (sub == 0) {
+                        free_ = ra == 0 || tc::mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1, &abort_flag, p.max_polls);
+                        if (!__all_sync(0xffffffffu, free_)) break;
+                        tc::tc_fence_after();
+                    }
+                    tc::tmem_st16(t_lane + (uint32_t)(sa * 32 * kSub + sub * 32), o0);
+                    tc::tmem_st16(t_lane + (uint32_t)(sa * 32 * kSub + sub * 32 + 16), o1);
                 }
-                bool free_ = ra == 0 || tc::mbar_wait_bounded(&a_empty[sa], (ra - 1) & 1, &abort_flag, p.max_polls);
                 if (!__all_sync(0xffffffffu, free_)) {
                     if (!abort_flag) fail(p.hdr, &abort_flag);
                     ok = false;
                     break;
                 }
-                tc::tc_fence_after();
-                tc::tmem_st16(t_lane + (uint32_t)(sa * 32), o0);
-                tc::tmem_st16(t_lane + (uint32_t)(sa * 32 + 16), o1);
                 tc::tmem_wait_st();
                 tc::tc_fence_before();
                 __syncwarp();
