@@ -182,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if ((int)blockIdx.x >= total) return;  // no tile for this CTA: nothing was taken yet
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sX = smem;                                // [kXStages][256 rows][128 B]
-    uint8_t* sQ = smem + kXStages * kXBytes;           // [kQStages][128 rows][64 B]
+    uint8_t* sX = smem;                                // [kXStages][kSub][256 rows][128 B]
+    uint8_t* sQ = smem + kXStages * kXBytes;           // [kQStages][kSub][128 rows][64 B]
     uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + kQStages * kQBytes);
     uint64_t* x_full = bars;                           // [kXStages] token tile landed (TMA bytes)
     uint64_t* x_empty = x_full + kXStages;             // [kXStages] MMAs reading it are done
