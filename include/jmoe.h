@@ -228,7 +228,7 @@ const char* jamba_moe_status_string(int status);
 /*
  * jamba_moe_debug_skip_copy — test hook for failure detection, off by default.  While `on` is
  * non-zero, the next forward calls on the tensor-core (prefill) path make CTA 0 of the W1/W3 GEMM
- * skip the copies of its second K step, with every pipeline wait bounded by a short poll limit:
+ * skip the copies of its second pipeline stage, with every wait bounded by a short poll limit:
  * the wait for those copies runs out, the kernel records JMOE_DEV_TIMEOUT in the workspace status
  * word, waits (bounded) for its other in-flight copies and MMAs, releases its tensor memory and
  * returns; the output of that call is not valid.  Nothing faults, traps or hangs, and the CUDA

@@ -104,7 +104,7 @@ struct Args {
     int band_max;         // token tiles per L2 band, at most
     int sched;            // which tile counter of the header this GEMM uses
     uint32_t max_polls;   // bound of every mbarrier wait
-    int skip_copy;        // test hook: CTA 0 skips the copies of the second K step of its first tile
+    int skip_copy;        // test hook: CTA 0 skips the copies of the second stage of its first tile
 };
 
 struct Tile {
@@ -720,7 +720,7 @@ cudaError_t launch_gemm2(WsHeader* hdr, const int32_t* perm, const uint16_t* h, 
 }  // namespace jmoe
 
 // Test hook: while `on` is non-zero, the W1/W3 tensor-core GEMM's CTA 0 skips the copies of the
-// second K step of its first tile, so the pipeline wait for them runs out (after a short bound)
+// second pipeline stage of its first tile, so the wait for them runs out (after a short bound)
 // and the kernel must report JMOE_DEV_TIMEOUT, release its resources and return.  Nothing faults
 // or hangs.
 extern "C" int jamba_moe_debug_skip_copy(int on) {
