@@ -229,8 +229,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32,
             }
         }
         // W2 with 16 tokens per pass: one k-step in flight per warp and 4 CTAs per SM stream faster
-        // than two steps at 2 CTAs per SM
-        gemv_pass<NT, kDual, kW8, (kW8 && ((!kDual && NT == 2) || NT == 4)) ? 1 : 2>(p, e, j0, rows, red);
+        // than two steps at 2 CTAs per SM; W1/W3 with 32 tokens per pass: one k-step (registers)
+        gemv_pass<NT, kDual, kW8, (kW8 && ((!kDual && NT == 2) || (kDual && NT == 4))) ? 1 : 2>(p, e, j0, rows, red);
         pdl_trigger();  // main loop done: the next kernel may start launching
         // epilogue over the totals: o = (mat, nt, lane', i); C fragment (lane' = 4g' + c'):
         // i = 0,1 -> row g', tokens 2c', 2c'+1; i = 2,3 -> row g'+8, same tokens.
